@@ -1,0 +1,167 @@
+/*
+ * saga.h -- C ABI of the SAGA + Atop-N single-token decode-attention library.
+ *
+ * Source of the operation: "More Value per Key: Asymmetric Sparse Attention for
+ * Faster LLM Decoding" (Elata et al.), cited as [MVK]:
+ *   scores     z_i = q . k_i / sqrt(d) over all cached positions, the current
+ *              token included                       [MVK] §2.1 Eq. (2), §2.2 Eq. (5)
+ *   selection  the N highest-scoring positions of each query head's score row
+ *              (Atop-N: compare each score against the N-th largest score; the
+ *              threshold is exact and recomputed on every call)
+ *                                                   [MVK] §2.5 Eq. (6), §3.1, App. C.1
+ *   softmax    over the selected logits only        [MVK] §3.1 Eq. (7), App. C.1
+ *   output     O = softmax(A[i]) V[i]               [MVK] §3.1 Eq. (7)
+ *   heads      SAGA decouples key heads h_k from value heads h_v; query head j
+ *              reads key head j / (h_q/h_k) and value head j / (h_q/h_v)
+ *              (contiguous blocks)                  [MVK] §3.2, §2.3, App. B Eq. (29)
+ * Ties at the N-th score go to the lowest position.  A row with L_b <= N
+ * selects all L_b positions (dense softmax attention).
+ *
+ * Layouts (all row-major, bf16 = IEEE bfloat16, device memory unless stated):
+ *   q         [B][h_q][d]            one query per head (decode, l_q = 1)
+ *   k_cache   [B][h_k][L_max][d]     positions 0..L_b-1 valid; the current token's
+ *   v_cache   [B][h_v][L_max][d]     key/value are already stored at L_b-1
+ *   seq_lens  int32 [B]              L_b, 1 <= L_b <= L_max
+ *   out       bf16 [B][h_q][d]       fp32 accumulation, one final round-to-nearest-even
+ *   sel_idx   int32 [B][h_q][N]      selected positions, ascending; -1 padding when L_b < N
+ *   sel_logit fp32  [B][h_q][N]      their scores z; -inf padding
+ *   scores    fp32  [B][h_q][stride] z for positions < L_b (stride >= L_max)
+ * B is the handle's current batch (saga_decode_set_batch; initially max_batch);
+ * L_max is the handle's max_seq_len, which is also the caches' position stride.
+ *
+ * Ownership: every tensor argument is caller-owned; the library never frees or
+ * retains it past the call.  The handle owns only its workspace (score rows,
+ * selection lists, statistics, staging), allocated once by saga_decode_init and
+ * released by saga_decode_free.  No call allocates memory, synchronises the
+ * stream or copies to the host, except saga_decode_status and the explicit
+ * host-buffer entry point saga_decode_attn_host (which copies but does not
+ * synchronise).  Calls run asynchronously, in order, on the handle's stream.
+ *
+ * Errors: every function returns an int code (SAGA_OK = 0).  Arguments are
+ * validated on the host before anything is enqueued; on error nothing runs.
+ * Data errors only the device can see (a seq_len outside [1, L_max]) zero that
+ * row's output, pad its selection and set a bit in the device status word,
+ * read and cleared by saga_decode_status.  Kernels never trap; every internal
+ * wait is bounded and reports SAGA_STATUS_TIMEOUT instead of hanging.
+ * A handle must not be used from two host threads at once.
+ *
+ * Limits: d in {64, 128}; h_k | h_q and h_v | h_q; g = h_q/h_k <= 64;
+ * 1 <= B <= max_batch <= 1024; 1 <= max_seq_len <= 2^24; 1 <= N <= max_N;
+ * max_batch * h_k * max_seq_len < 2^31.  Needs a compute capability 10.0 GPU
+ * (B200, sm_100a).
+ */
+#ifndef SAGA_H
+#define SAGA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define SAGA_OK               0
+#define SAGA_ERR_INVALID_ARG  1  /* null pointer, bad size, mismatched heads, N > max_N ... */
+#define SAGA_ERR_UNSUPPORTED  2  /* valid but not built: d not in {64,128}, g > 64, wrong GPU */
+#define SAGA_ERR_CUDA         3  /* a CUDA runtime/driver call failed */
+#define SAGA_ERR_DEVICE       4  /* saga_decode_status found an error bit set */
+
+/* Device status bits (saga_decode_status). */
+#define SAGA_STATUS_BAD_SEQ_LEN   0x1   /* some seq_lens[b] outside [1, L_max]: row zeroed */
+#define SAGA_STATUS_TIMEOUT       0x2   /* an internal pipeline wait ran out: results invalid */
+#define SAGA_STATUS_INFO_EXACT_FALLBACK 0x100  /* informational: a row needed the full radix
+                                                   select (very flat score rows); not an error */
+
+typedef struct saga_ctx* saga_handle;
+
+/* Create a handle and its workspace for caches of up to max_batch rows of
+ * max_seq_len positions, with h_q query, h_k key and h_v value heads of size
+ * head_dim, and selections of up to max_N positions.  cuda_stream is a
+ * cudaStream_t (NULL = legacy default stream).  The current CUDA device at
+ * this call is the handle's device.  Workspace: about
+ * 4*max_batch*h_q*(round_up(max_seq_len,32) + 2*max_N + 2) bytes.
+ * Returns SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_CUDA. */
+int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len,
+                     int h_q, int h_k, int h_v, int head_dim, int max_N,
+                     void* cuda_stream);
+
+/* Set the batch B (1 <= B <= max_batch) used by later calls. */
+int saga_decode_set_batch(saga_handle h, int batch);
+
+/* Set the stream later calls are enqueued on (a cudaStream_t). */
+int saga_decode_set_stream(saga_handle h, void* cuda_stream);
+
+/* The decode step ([MVK] Eqs. (2), (5)-(7)): scores, exact top-N selection per
+ * query head, softmax over the selection and the gathered P.V, for every
+ * (b, j).  q, k_cache, v_cache, seq_lens, out: device pointers (layouts above).
+ * h_q, h_k, h_v, head_dim must equal the handle's; 1 <= N <= max_N. */
+int saga_decode_attn(saga_handle h, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* seq_lens,
+                     int h_q, int h_k, int h_v, int head_dim, int N, void* out);
+
+/* As saga_decode_attn, and also writes the selection: sel_idx / sel_logit are
+ * device arrays [B][h_q][N] (either may be NULL). */
+int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* seq_lens,
+                        int h_q, int h_k, int h_v, int head_dim, int N, void* out,
+                        int32_t* sel_idx, float* sel_logit);
+
+/* The decode step with the per-step inputs and result in HOST memory:
+ * q_host (bf16 [B][h_q][d]) and seq_lens_host (int32 [B]) are copied to the
+ * handle's device staging, the step runs, and the result is copied back to
+ * out_host (bf16 [B][h_q][d]).  The caches stay in device memory (they are the
+ * resident KV cache).  All three copies are enqueued asynchronously on the
+ * handle's stream: host buffers should be pinned, and out_host is valid only
+ * after the stream is synchronised (e.g. by saga_decode_status). */
+int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache,
+                          const void* v_cache, const int32_t* seq_lens_host,
+                          int h_q, int h_k, int h_v, int head_dim, int N,
+                          void* out_host);
+
+/* Stage S1 alone ([MVK] Eq. (2), (5)): scores[b][j][i] = q[b][j] . k[b][j/g][i]
+ * / sqrt(d) for i < L_b, fp32, into the caller's array with row stride
+ * scores_stride >= L_max (entries i >= L_b are not written). */
+int saga_score(saga_handle h, const void* q, const void* k_cache,
+               const int32_t* seq_lens, int h_q, int h_k, int head_dim,
+               float* scores, int scores_stride);
+
+/* Stage S2 alone ([MVK] Eq. (6), App. C.1): exact top-N selection of each
+ * caller-given fp32 score row (layout of saga_score), ties to the lowest
+ * position; writes sel_idx and sel_logit ([B][h_q][N], non-NULL). */
+int saga_select(saga_handle h, const float* scores, int scores_stride,
+                const int32_t* seq_lens, int h_q, int N,
+                int32_t* sel_idx, float* sel_logit);
+
+/* Stages S3+S4 alone ([MVK] Eq. (7)): softmax over the valid entries of each
+ * selection row (sel_idx >= 0) and the gathered P.V over v_cache, bf16 out. */
+int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
+                 const void* v_cache, const int32_t* seq_lens, int h_q, int h_v,
+                 int head_dim, int N, void* out);
+
+/* Synchronise the handle's stream, then return (in *device_status) and clear
+ * the device status word.  Returns SAGA_ERR_DEVICE if an error bit
+ * (SAGA_STATUS_BAD_SEQ_LEN or SAGA_STATUS_TIMEOUT) was set, else SAGA_OK. */
+int saga_decode_status(saga_handle h, int* device_status);
+
+/* Total number of kernels this handle has launched. */
+int saga_decode_launch_count(saga_handle h, long long* count);
+
+/* Profiling: when enabled, each decode call records CUDA events around its
+ * score kernel and around the whole call on the handle's stream (up to
+ * max_calls calls).  saga_decode_profile_read synchronises and returns the
+ * summed milliseconds and the number of calls recorded, then resets. */
+int saga_decode_profile(saga_handle h, int enable, int max_calls);
+int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms,
+                             int* n_calls);
+
+/* A static description of a return code. */
+const char* saga_decode_error_string(int code);
+
+/* Release the handle and its workspace (synchronises its stream first). */
+int saga_decode_free(saga_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGA_H */
