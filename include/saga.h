@@ -55,6 +55,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define SAGA_API __attribute__((visibility("default")))
+#else
+#define SAGA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -69,6 +75,7 @@ extern "C" {
 /* Device status bits (saga_decode_status). */
 #define SAGA_STATUS_BAD_SEQ_LEN   0x1   /* some seq_lens[b] outside [1, L_max]: row zeroed */
 #define SAGA_STATUS_TIMEOUT       0x2   /* an internal pipeline wait ran out: results invalid */
+#define SAGA_STATUS_BAD_INDEX     0x4   /* saga_combine got an index >= L_b: that slot ignored */
 #define SAGA_STATUS_INFO_EXACT_FALLBACK 0x100  /* informational: a row needed the full radix
                                                    select (very flat score rows); not an error */
 
@@ -81,27 +88,27 @@ typedef struct saga_ctx* saga_handle;
  * this call is the handle's device.  Workspace: about
  * 4*max_batch*h_q*(round_up(max_seq_len,32) + 2*max_N + 2) bytes.
  * Returns SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_CUDA. */
-int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len,
+SAGA_API int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len,
                      int h_q, int h_k, int h_v, int head_dim, int max_N,
                      void* cuda_stream);
 
 /* Set the batch B (1 <= B <= max_batch) used by later calls. */
-int saga_decode_set_batch(saga_handle h, int batch);
+SAGA_API int saga_decode_set_batch(saga_handle h, int batch);
 
 /* Set the stream later calls are enqueued on (a cudaStream_t). */
-int saga_decode_set_stream(saga_handle h, void* cuda_stream);
+SAGA_API int saga_decode_set_stream(saga_handle h, void* cuda_stream);
 
 /* The decode step ([MVK] Eqs. (2), (5)-(7)): scores, exact top-N selection per
  * query head, softmax over the selection and the gathered P.V, for every
  * (b, j).  q, k_cache, v_cache, seq_lens, out: device pointers (layouts above).
  * h_q, h_k, h_v, head_dim must equal the handle's; 1 <= N <= max_N. */
-int saga_decode_attn(saga_handle h, const void* q, const void* k_cache,
+SAGA_API int saga_decode_attn(saga_handle h, const void* q, const void* k_cache,
                      const void* v_cache, const int32_t* seq_lens,
                      int h_q, int h_k, int h_v, int head_dim, int N, void* out);
 
 /* As saga_decode_attn, and also writes the selection: sel_idx / sel_logit are
  * device arrays [B][h_q][N] (either may be NULL). */
-int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cache,
+SAGA_API int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cache,
                         const void* v_cache, const int32_t* seq_lens,
                         int h_q, int h_k, int h_v, int head_dim, int N, void* out,
                         int32_t* sel_idx, float* sel_logit);
@@ -113,7 +120,7 @@ int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cache,
  * resident KV cache).  All three copies are enqueued asynchronously on the
  * handle's stream: host buffers should be pinned, and out_host is valid only
  * after the stream is synchronised (e.g. by saga_decode_status). */
-int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache,
+SAGA_API int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache,
                           const void* v_cache, const int32_t* seq_lens_host,
                           int h_q, int h_k, int h_v, int head_dim, int N,
                           void* out_host);
@@ -121,44 +128,47 @@ int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache
 /* Stage S1 alone ([MVK] Eq. (2), (5)): scores[b][j][i] = q[b][j] . k[b][j/g][i]
  * / sqrt(d) for i < L_b, fp32, into the caller's array with row stride
  * scores_stride >= L_max (entries i >= L_b are not written). */
-int saga_score(saga_handle h, const void* q, const void* k_cache,
+SAGA_API int saga_score(saga_handle h, const void* q, const void* k_cache,
                const int32_t* seq_lens, int h_q, int h_k, int head_dim,
                float* scores, int scores_stride);
 
 /* Stage S2 alone ([MVK] Eq. (6), App. C.1): exact top-N selection of each
  * caller-given fp32 score row (layout of saga_score), ties to the lowest
  * position; writes sel_idx and sel_logit ([B][h_q][N], non-NULL). */
-int saga_select(saga_handle h, const float* scores, int scores_stride,
+SAGA_API int saga_select(saga_handle h, const float* scores, int scores_stride,
                 const int32_t* seq_lens, int h_q, int N,
                 int32_t* sel_idx, float* sel_logit);
 
 /* Stages S3+S4 alone ([MVK] Eq. (7)): softmax over the valid entries of each
- * selection row (sel_idx >= 0) and the gathered P.V over v_cache, bf16 out. */
-int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
+ * selection row ([B][h_q][N]; entries with sel_idx < 0 are padding, entries
+ * >= L_b are ignored and flagged SAGA_STATUS_BAD_INDEX) and the gathered P.V
+ * over v_cache, bf16 out.  A row with no valid entry gets zeros. */
+SAGA_API int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
                  const void* v_cache, const int32_t* seq_lens, int h_q, int h_v,
                  int head_dim, int N, void* out);
 
 /* Synchronise the handle's stream, then return (in *device_status) and clear
  * the device status word.  Returns SAGA_ERR_DEVICE if an error bit
- * (SAGA_STATUS_BAD_SEQ_LEN or SAGA_STATUS_TIMEOUT) was set, else SAGA_OK. */
-int saga_decode_status(saga_handle h, int* device_status);
+ * (SAGA_STATUS_BAD_SEQ_LEN, SAGA_STATUS_TIMEOUT or SAGA_STATUS_BAD_INDEX) was
+ * set, else SAGA_OK. */
+SAGA_API int saga_decode_status(saga_handle h, int* device_status);
 
 /* Total number of kernels this handle has launched. */
-int saga_decode_launch_count(saga_handle h, long long* count);
+SAGA_API int saga_decode_launch_count(saga_handle h, long long* count);
 
 /* Profiling: when enabled, each decode call records CUDA events around its
  * score kernel and around the whole call on the handle's stream (up to
  * max_calls calls).  saga_decode_profile_read synchronises and returns the
  * summed milliseconds and the number of calls recorded, then resets. */
-int saga_decode_profile(saga_handle h, int enable, int max_calls);
-int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms,
+SAGA_API int saga_decode_profile(saga_handle h, int enable, int max_calls);
+SAGA_API int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms,
                              int* n_calls);
 
 /* A static description of a return code. */
-const char* saga_decode_error_string(int code);
+SAGA_API const char* saga_decode_error_string(int code);
 
 /* Release the handle and its workspace (synchronises its stream first). */
-int saga_decode_free(saga_handle h);
+SAGA_API int saga_decode_free(saga_handle h);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,494 @@
+// saga_api.cu -- the C ABI declared in include/saga.h: argument validation,
+// the handle and its workspace, TMA descriptor encoding and the launch plan.
+//
+// One decode call enqueues two kernels on the handle's stream:
+//   score_kernel          S1, persistent, one CTA per SM (tcgen05 + TMA)
+//   select_combine_kernel S2-S4, one CTA per (batch row, query head)
+// Nothing is allocated, synchronised or copied to the host on that path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "saga.h"
+#include "ptx.cuh"
+#include "score_kernel.cuh"
+#include "select_kernel.cuh"
+
+using namespace saga;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), box {64, box_rows}, 128-byte swizzle.
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+struct saga_ctx {
+  int device = 0;
+  int num_sms = 0;
+  int max_batch = 0, batch = 0, max_seq_len = 0, h_q = 0, h_k = 0, h_v = 0, d = 0, max_N = 0;
+  int g = 0, g_v = 0, npad = 0;
+  long long z_stride = 0;
+  cudaStream_t stream = nullptr;
+  // workspace (one allocation)
+  void* ws = nullptr;
+  float* z = nullptr;
+  uint32_t* stat_min = nullptr;
+  uint32_t* stat_max = nullptr;
+  int32_t* sel_idx = nullptr;
+  float* sel_logit = nullptr;
+  int* status = nullptr;
+  __nv_bfloat16* q_stage = nullptr;
+  __nv_bfloat16* out_stage = nullptr;
+  int32_t* lens_stage = nullptr;
+  long long launches = 0;
+  // profiling
+  bool prof = false;
+  int prof_max = 0, prof_n = 0;
+  std::vector<cudaEvent_t> ev;   // 3 per recorded call: start, after score, end
+};
+
+namespace {
+
+int set_smem_attrs_once() {
+  static int rc = -1;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    cudaError_t e = cudaSuccess;
+#define SAGA_ATTR(D, NP)                                                                       \
+  if (e == cudaSuccess)                                                                        \
+    e = cudaFuncSetAttribute(score_kernel<D, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             ScoreShape<D, NP>::kSmemBytes);
+    SAGA_ATTR(64, 16) SAGA_ATTR(64, 32) SAGA_ATTR(64, 48) SAGA_ATTR(64, 64)
+    SAGA_ATTR(128, 16) SAGA_ATTR(128, 32) SAGA_ATTR(128, 48) SAGA_ATTR(128, 64)
+#undef SAGA_ATTR
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(select_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(SelectSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(select_combine_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(SelectSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(SelectSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(combine_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(SelectSmem)));
+    rc = (e == cudaSuccess) ? 0 : 1;
+  });
+  return rc;
+}
+
+template <int D, int NP>
+cudaError_t launch_score_t(saga_ctx* h, const CUtensorMap& mk, const CUtensorMap& mq,
+                           const ScoreParams& p, int grid) {
+  score_kernel<D, NP><<<grid, kScoreThreads, ScoreShape<D, NP>::kSmemBytes, h->stream>>>(mk, mq, p);
+  return cudaGetLastError();
+}
+
+int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
+                 float* z, long long z_stride, bool stats) {
+  CUtensorMap mk, mq;
+  const uint64_t k_rows = static_cast<uint64_t>(h->batch) * h->h_k * h->max_seq_len;
+  const uint64_t q_rows = static_cast<uint64_t>(h->batch) * h->h_q;
+  if (!encode_bf16_2d(&mk, k_cache, k_rows, h->d, kTileM)) return SAGA_ERR_CUDA;
+  if (!encode_bf16_2d(&mq, q, q_rows, h->d, h->npad)) return SAGA_ERR_CUDA;
+  ScoreParams p;
+  p.seq_lens = seq_lens;
+  p.z = z;
+  p.stat_min = stats ? h->stat_min : nullptr;
+  p.stat_max = stats ? h->stat_max : nullptr;
+  p.status = h->status;
+  p.B = h->batch;
+  p.h_q = h->h_q;
+  p.h_k = h->h_k;
+  p.g = h->g;
+  p.L_max = h->max_seq_len;
+  p.z_stride = z_stride;
+  p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d)));
+  const long long max_units =
+      static_cast<long long>(h->batch) * h->h_k * ((h->max_seq_len + kTileM - 1) / kTileM);
+  const int grid = static_cast<int>(max_units < h->num_sms ? max_units : h->num_sms);
+  cudaError_t e = cudaErrorInvalidValue;
+#define SAGA_CASE(D, NP) \
+  if (h->d == D && h->npad == NP) e = launch_score_t<D, NP>(h, mk, mq, p, grid);
+  SAGA_CASE(64, 16) SAGA_CASE(64, 32) SAGA_CASE(64, 48) SAGA_CASE(64, 64)
+  SAGA_CASE(128, 16) SAGA_CASE(128, 32) SAGA_CASE(128, 48) SAGA_CASE(128, 64)
+#undef SAGA_CASE
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  ++h->launches;
+  return SAGA_OK;
+}
+
+int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
+                  const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_logit,
+                  const void* v_cache, void* out) {
+  SelectParams p;
+  p.z = z;
+  p.z_stride = z_stride;
+  p.stat_min = stats ? h->stat_min : nullptr;
+  p.stat_max = stats ? h->stat_max : nullptr;
+  p.seq_lens = seq_lens;
+  p.B = h->batch;
+  p.h_q = h->h_q;
+  p.L_max = h->max_seq_len;
+  p.N = N;
+  p.z_vec4 = ((z_stride % 4) == 0 && (reinterpret_cast<uintptr_t>(z) % 16) == 0) ? 1 : 0;
+  p.sel_idx = sel_idx;
+  p.sel_logit = sel_logit;
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.h_v = h->h_v;
+  p.g_v = h->g_v;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = h->status;
+  const int grid = h->batch * h->h_q;
+  const size_t smem = sizeof(SelectSmem);
+  if (h->d == 64)
+    select_combine_kernel<64><<<grid, kSelThreads, smem, h->stream>>>(p);
+  else
+    select_combine_kernel<128><<<grid, kSelThreads, smem, h->stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+  ++h->launches;
+  return SAGA_OK;
+}
+
+int check_heads(saga_ctx* h, int h_q, int h_k, int h_v, int d) {
+  if (h_q != h->h_q || h_k != h->h_k || h_v != h->h_v || d != h->d) return SAGA_ERR_INVALID_ARG;
+  return SAGA_OK;
+}
+
+struct DeviceGuard {   // run a call on the handle's device, restore the caller's
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* seq_lens, int N, void* out, int32_t* sel_idx, float* sel_logit) {
+  if (!q || !k_cache || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  const bool prof = h->prof && h->prof_n < h->prof_max;
+  cudaEvent_t* ev = prof ? &h->ev[3 * h->prof_n] : nullptr;
+  if (prof && cudaEventRecord(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  int rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true);
+  if (rc) return rc;
+  if (prof && cudaEventRecord(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  // The selection goes to the caller's arrays when given, else to the workspace
+  // (row stride N either way).
+  int32_t* si = sel_idx ? sel_idx : h->sel_idx;
+  float* sl = sel_logit ? sel_logit : h->sel_logit;
+  rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl, v_cache, out);
+  if (rc) return rc;
+  if (prof) {
+    if (cudaEventRecord(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    ++h->prof_n;
+  }
+  return SAGA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* saga_decode_error_string(int code) {
+  switch (code) {
+    case SAGA_OK: return "ok";
+    case SAGA_ERR_INVALID_ARG: return "invalid argument";
+    case SAGA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case SAGA_ERR_CUDA: return "CUDA call failed";
+    case SAGA_ERR_DEVICE: return "device reported an error (see saga_decode_status)";
+    default: return "unknown error code";
+  }
+}
+
+int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_q, int h_k,
+                     int h_v, int head_dim, int max_N, void* cuda_stream) {
+  if (!handle) return SAGA_ERR_INVALID_ARG;
+  *handle = nullptr;
+  if (max_batch < 1 || max_batch > kMaxBatch) return SAGA_ERR_INVALID_ARG;
+  if (max_seq_len < 1 || max_seq_len > (1 << 24)) return SAGA_ERR_INVALID_ARG;
+  if (h_q < 1 || h_k < 1 || h_v < 1 || max_N < 1) return SAGA_ERR_INVALID_ARG;
+  if (h_q % h_k != 0 || h_q % h_v != 0) return SAGA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_batch) * h_k * max_seq_len >= (1ll << 31)) return SAGA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_batch) * h_q > (1ll << 30)) return SAGA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return SAGA_ERR_UNSUPPORTED;
+  const int g = h_q / h_k;
+  if (g > 64) return SAGA_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGA_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (prop.major != 10) return SAGA_ERR_UNSUPPORTED;
+  if (set_smem_attrs_once() != 0) return SAGA_ERR_CUDA;
+  if (!get_encode_fn()) return SAGA_ERR_CUDA;
+
+  saga_ctx* h = new (std::nothrow) saga_ctx();
+  if (!h) return SAGA_ERR_CUDA;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->max_batch = h->batch = max_batch;
+  h->max_seq_len = max_seq_len;
+  h->h_q = h_q; h->h_k = h_k; h->h_v = h_v; h->d = head_dim; h->max_N = max_N;
+  h->g = g; h->g_v = h_q / h_v;
+  h->npad = round_up(g, 16);
+  h->z_stride = round_up(max_seq_len, 32);
+  h->stream = static_cast<cudaStream_t>(cuda_stream);
+
+  const size_t rows = static_cast<size_t>(max_batch) * h_q;
+  const size_t z_bytes = rows * h->z_stride * sizeof(float);
+  const size_t stat_bytes = rows * sizeof(uint32_t);
+  const size_t sel_bytes = rows * static_cast<size_t>(max_N) * 4;
+  const size_t qo_bytes = rows * head_dim * 2;
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t total = al(z_bytes) + 2 * al(stat_bytes) + 2 * al(sel_bytes) + al(256) +
+                       2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4);
+  if (cudaMalloc(&h->ws, total) != cudaSuccess) { delete h; return SAGA_ERR_CUDA; }
+  uint8_t* w = static_cast<uint8_t*>(h->ws);
+  h->z = reinterpret_cast<float*>(w); w += al(z_bytes);
+  h->stat_min = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
+  h->stat_max = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
+  h->sel_idx = reinterpret_cast<int32_t*>(w); w += al(sel_bytes);
+  h->sel_logit = reinterpret_cast<float*>(w); w += al(sel_bytes);
+  h->status = reinterpret_cast<int*>(w); w += al(256);
+  h->q_stage = reinterpret_cast<__nv_bfloat16*>(w); w += al(qo_bytes);
+  h->out_stage = reinterpret_cast<__nv_bfloat16*>(w); w += al(qo_bytes);
+  h->lens_stage = reinterpret_cast<int32_t*>(w);
+  if (cudaMemset(h->stat_min, 0xFF, stat_bytes) != cudaSuccess ||
+      cudaMemset(h->stat_max, 0x00, stat_bytes) != cudaSuccess ||
+      cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(h->ws);
+    delete h;
+    return SAGA_ERR_CUDA;
+  }
+  *handle = h;
+  return SAGA_OK;
+}
+
+int saga_decode_set_batch(saga_handle h, int batch) {
+  if (!h || batch < 1 || batch > h->max_batch) return SAGA_ERR_INVALID_ARG;
+  h->batch = batch;
+  return SAGA_OK;
+}
+
+int saga_decode_set_stream(saga_handle h, void* cuda_stream) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  h->stream = static_cast<cudaStream_t>(cuda_stream);
+  return SAGA_OK;
+}
+
+int saga_decode_attn(saga_handle h, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* seq_lens, int h_q, int h_k, int h_v, int head_dim, int N,
+                     void* out) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, nullptr, nullptr);
+}
+
+int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* seq_lens, int h_q, int h_k, int h_v, int head_dim, int N,
+                        void* out, int32_t* sel_idx, float* sel_logit) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit);
+}
+
+int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache,
+                          const void* v_cache, const int32_t* seq_lens_host, int h_q, int h_k,
+                          int h_v, int head_dim, int N, void* out_host) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  if (!q_host || !seq_lens_host || !out_host || !k_cache || !v_cache) return SAGA_ERR_INVALID_ARG;
+  if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  const size_t qo = static_cast<size_t>(h->batch) * h->h_q * h->d * 2;
+  if (cudaMemcpyAsync(h->q_stage, q_host, qo, cudaMemcpyHostToDevice, h->stream) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+  if (cudaMemcpyAsync(h->lens_stage, seq_lens_host, static_cast<size_t>(h->batch) * 4,
+                      cudaMemcpyHostToDevice, h->stream) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+  int rc = decode_impl(h, h->q_stage, k_cache, v_cache, h->lens_stage, N, h->out_stage,
+                       nullptr, nullptr);
+  if (rc) return rc;
+  if (cudaMemcpyAsync(out_host, h->out_stage, qo, cudaMemcpyDeviceToHost, h->stream) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+  return SAGA_OK;
+}
+
+int saga_score(saga_handle h, const void* q, const void* k_cache, const int32_t* seq_lens,
+               int h_q, int h_k, int head_dim, float* scores, int scores_stride) {
+  if (!h || !q || !k_cache || !seq_lens || !scores) return SAGA_ERR_INVALID_ARG;
+  if (h_q != h->h_q || h_k != h->h_k || head_dim != h->d) return SAGA_ERR_INVALID_ARG;
+  if (scores_stride < h->max_seq_len) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  return launch_score(h, q, k_cache, seq_lens, scores, scores_stride, false);
+}
+
+int saga_select(saga_handle h, const float* scores, int scores_stride, const int32_t* seq_lens,
+                int h_q, int N, int32_t* sel_idx, float* sel_logit) {
+  if (!h || !scores || !seq_lens || !sel_idx || !sel_logit) return SAGA_ERR_INVALID_ARG;
+  if (h_q != h->h_q || scores_stride < h->max_seq_len) return SAGA_ERR_INVALID_ARG;
+  if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  return launch_select(h, scores, scores_stride, false, seq_lens, N, sel_idx, sel_logit,
+                       nullptr, nullptr);
+}
+
+int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
+                 const void* v_cache, const int32_t* seq_lens, int h_q, int h_v, int head_dim,
+                 int N, void* out) {
+  if (!h || !sel_idx || !sel_logit || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (h_q != h->h_q || h_v != h->h_v || head_dim != h->d) return SAGA_ERR_INVALID_ARG;
+  if (N < 1) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  SelectParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.seq_lens = seq_lens;
+  p.B = h->batch;
+  p.h_q = h->h_q;
+  p.L_max = h->max_seq_len;
+  p.N = N;
+  p.sel_idx = const_cast<int32_t*>(sel_idx);
+  p.sel_logit = const_cast<float*>(sel_logit);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.h_v = h->h_v;
+  p.g_v = h->g_v;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = h->status;
+  const int grid = h->batch * h->h_q;
+  const size_t smem = sizeof(SelectSmem);
+  if (h->d == 64)
+    combine_kernel<64><<<grid, kSelThreads, smem, h->stream>>>(p);
+  else
+    combine_kernel<128><<<grid, kSelThreads, smem, h->stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+  ++h->launches;
+  return SAGA_OK;
+}
+
+int saga_decode_status(saga_handle h, int* device_status) {
+  if (!h || !device_status) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  int v = 0;
+  if (cudaStreamSynchronize(h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+  if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SAGA_ERR_CUDA;
+  *device_status = v;
+  return (v & (SAGA_STATUS_BAD_SEQ_LEN | SAGA_STATUS_TIMEOUT | SAGA_STATUS_BAD_INDEX))
+             ? SAGA_ERR_DEVICE : SAGA_OK;
+}
+
+int saga_decode_launch_count(saga_handle h, long long* count) {
+  if (!h || !count) return SAGA_ERR_INVALID_ARG;
+  *count = h->launches;
+  return SAGA_OK;
+}
+
+int saga_decode_profile(saga_handle h, int enable, int max_calls) {
+  if (!h || (enable && max_calls < 1)) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+  h->ev.clear();
+  h->prof = false;
+  h->prof_n = 0;
+  h->prof_max = 0;
+  if (!enable) return SAGA_OK;
+  h->ev.resize(3 * static_cast<size_t>(max_calls));
+  for (auto& e : h->ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return SAGA_ERR_CUDA;
+  h->prof_max = max_calls;
+  h->prof = true;
+  return SAGA_OK;
+}
+
+int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms, int* n_calls) {
+  if (!h || !score_ms || !call_ms || !n_calls) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  if (cudaStreamSynchronize(h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  double s = 0.0, c = 0.0;
+  for (int i = 0; i < h->prof_n; ++i) {
+    float a = 0.0f, b = 0.0f;
+    if (cudaEventElapsedTime(&a, h->ev[3 * i], h->ev[3 * i + 1]) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (cudaEventElapsedTime(&b, h->ev[3 * i], h->ev[3 * i + 2]) != cudaSuccess) return SAGA_ERR_CUDA;
+    s += a;
+    c += b;
+  }
+  *score_ms = s;
+  *call_ms = c;
+  *n_calls = h->prof_n;
+  h->prof_n = 0;
+  return SAGA_OK;
+}
+
+int saga_decode_free(saga_handle h) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  int rc = SAGA_OK;
+  {
+    DeviceGuard dg(h->device);
+    if (h->stream && cudaStreamSynchronize(h->stream) != cudaSuccess) rc = SAGA_ERR_CUDA;
+    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    if (h->ws && cudaFree(h->ws) != cudaSuccess) rc = SAGA_ERR_CUDA;
+  }
+  delete h;
+  return rc;
+}
+
+}  // extern "C"

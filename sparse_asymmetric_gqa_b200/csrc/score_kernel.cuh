@@ -1,0 +1,309 @@
+// score_kernel.cuh -- S1, the score pass: z[b, j, i] = q[b, j] . K[b, j/g, i] / sqrt(d)
+// ("More Value per Key", §2.1 Eq. (2) and §2.2 Eq. (5)), for every cached
+// position i < L_b of every query head j.
+//
+// Shape of the work: for one (batch row b, key head kh) the g query heads that
+// share the key head form a [g x d] matrix Q and the cache a [L_b x d] matrix
+// K, so the scores are the skinny product K . Q^T.  The K stream is the whole
+// cost (g flop per byte), so the kernel is built to move K at HBM speed and to
+// read every K row exactly once for all g heads:
+//
+//   * persistent CTAs, one per SM, each owning a contiguous range of 128-row
+//     tiles of the flattened (b, kh, tile) space (ragged seq_lens balanced);
+//   * warp 0 streams K tiles (and the group's q rows) into a ring of shared
+//     memory stages with TMA (128-byte swizzle, L2 evict-first for K);
+//   * warp 1 issues tcgen05.mma (M = 128 positions, N = g padded to 16k,
+//     K = 16 per instruction) into a double-buffered TMEM accumulator;
+//   * warps 2-5 read the accumulator back with tcgen05.ld (thread = position,
+//     registers = heads), scale, store z row-wise (coalesced per head) and keep
+//     per-(b, j) min/max statistics for the selector's first pass.
+#pragma once
+
+#include <cuda.h>
+#include "ptx.cuh"
+
+namespace saga {
+
+constexpr int kTileM = 128;          // positions per tile (MMA M)
+constexpr int kScoreThreads = 192;   // 6 warps: TMA, MMA, 4 x epilogue
+constexpr int kMaxBatch = 1024;
+
+struct ScoreParams {
+  const int32_t* seq_lens;   // [B]
+  float* z;                  // [B*h_q][z_stride]
+  uint32_t* stat_min;        // [B*h_q] ordered keys, or nullptr
+  uint32_t* stat_max;
+  int* status;
+  int B, h_q, h_k, g, L_max;
+  long long z_stride;
+  float scale;               // 1/sqrt(d), rounded to fp32
+};
+
+template <int D, int NPAD>
+struct ScoreShape {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(NPAD % 16 == 0 && NPAD >= 16 && NPAD <= 64, "padded group");
+  static constexpr int kParts = D / 64;                 // 128-byte swizzle atoms along d
+  static constexpr int kAPart = kTileM * 128;           // 16 KB of K per atom
+  static constexpr int kBPart = NPAD * 128;             // q rows per atom
+  static constexpr int kStageBytes = kParts * (kAPart + kBPart);
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw < 8 ? kStagesRaw : 8;
+  static constexpr int kTmemCols = (2 * NPAD <= 32) ? 32 : ((2 * NPAD <= 64) ? 64 : 128);
+  static constexpr int kAccStride = kTmemCols / 2;      // column offset of accumulator 1
+  static constexpr int kNumBars = 2 * kStages + 5;      // full, empty, accf[2], acce[2], drain
+  static constexpr int kCtrlBytes = kNumBars * 8 + 16 + 2 * (kMaxBatch + 1) * 4;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kCtrlBytes;
+  static_assert(kStages >= 2, "stages");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+};
+
+// Walks the flattened (b, kh, tile) space of one CTA in order.
+struct TileCursor {
+  int b, kh, t, tiles, Lb;
+  __device__ void seek(long long u, const int* unit_off, const int* lens, int B, int h_k) {
+    int lo = 0, hi = B;                       // largest b with unit_off[b] <= u
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (unit_off[mid] <= u) lo = mid; else hi = mid;
+    }
+    b = lo;
+    while (b < B && unit_off[b + 1] <= u) ++b;  // skip rows without tiles
+    Lb = (b < B) ? lens[b] : 0;
+    tiles = (Lb + kTileM - 1) / kTileM;
+    const long long r = u - unit_off[b];
+    kh = tiles ? static_cast<int>(r / tiles) : 0;
+    t = tiles ? static_cast<int>(r % tiles) : 0;
+  }
+  __device__ void next(const int* unit_off, const int* lens, int B, int h_k) {
+    if (++t < tiles) return;
+    t = 0;
+    if (++kh < h_k) return;
+    kh = 0;
+    do { ++b; } while (b < B && unit_off[b + 1] == unit_off[b]);
+    Lb = (b < B) ? lens[b] : 0;
+    tiles = (Lb + kTileM - 1) / kTileM;
+  }
+};
+
+__device__ __forceinline__ void st_global_hint(float* p, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" :: "l"(p), "f"(v), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
+  *abort_flag = 1;
+  atomicOr(status, 0x2 /* SAGA_STATUS_TIMEOUT */);
+}
+
+template <int D, int NPAD>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+score_kernel(const __grid_constant__ CUtensorMap tmap_k,
+             const __grid_constant__ CUtensorMap tmap_q, const ScoreParams p) {
+  using S = ScoreShape<D, NPAD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kStages * S::kStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* lens = reinterpret_cast<int*>(tmem_slot + 4);
+  int* unit_off = lens + kMaxBatch;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_addr(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S::kStages + s); };
+  auto accf_bar = [&](int i) { return bar0 + 8u * (2 * S::kStages + i); };
+  auto acce_bar = [&](int i) { return bar0 + 8u * (2 * S::kStages + 2 + i); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * S::kStages + 4);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < S::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+      for (int i = 0; i < 2; ++i) { mbar_init(accf_bar(i), 1); mbar_init(acce_bar(i), 4); }
+      mbar_init(drain_bar, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_q);
+    }
+    // Tile counts per batch row: h_k * ceil(L_b / 128) for a valid L_b, else 0.
+    int carry = 0;
+    for (int b0 = 0; b0 < p.B; b0 += 32) {
+      const int b = b0 + lane;
+      int L = 0, units = 0;
+      if (b < p.B) {
+        L = p.seq_lens[b];
+        if (L < 1 || L > p.L_max) L = 0;
+        units = p.h_k * ((L + kTileM - 1) / kTileM);
+        lens[b] = L;
+      }
+      int incl = units;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b == 0) unit_off[0] = 0;
+      if (b < p.B) unit_off[b + 1] = carry + incl;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const long long total = unit_off[p.B];
+  const long long u0 = total * blockIdx.x / gridDim.x;
+  const long long u1 = total * (blockIdx.x + 1) / gridDim.x;
+  const int n_tiles = static_cast<int>(u1 - u0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      const uint64_t pol_k = policy_evict_first();
+      const uint64_t pol_q = policy_evict_last();
+      TileCursor c;
+      c.seek(u0, unit_off, lens, p.B, p.h_k);
+      int i = 0;
+      for (; i < n_tiles; ++i) {
+        const int s = i % S::kStages;
+        const uint32_t ph = (i / S::kStages) & 1;
+        if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag)) { raise_abort(abort_flag, p.status); break; }
+        mbar_arrive_expect_tx(full_bar(s), S::kStageBytes);
+        const int row = (c.b * p.h_k + c.kh) * p.L_max + c.t * kTileM;
+        const int qrow = c.b * p.h_q + c.kh * p.g;
+        const uint32_t a = smem_addr(stages + s * S::kStageBytes);
+        const uint32_t bq = a + S::kParts * S::kAPart;
+#pragma unroll
+        for (int part = 0; part < S::kParts; ++part)
+          tma_load_2d(a + part * S::kAPart, &tmap_k, part * 64, row, full_bar(s), pol_k);
+#pragma unroll
+        for (int part = 0; part < S::kParts; ++part)
+          tma_load_2d(bq + part * S::kBPart, &tmap_q, part * 64, qrow, full_bar(s), pol_q);
+        c.next(unit_off, lens, p.B, p.h_k);
+      }
+      // Let every load this thread issued land before the CTA can exit.
+      const int first = i > S::kStages ? i - S::kStages : 0;
+      for (int k = first; k < i; ++k) {
+        volatile int never = 0;
+        mbar_wait(full_bar(k % S::kStages), (k / S::kStages) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileM, NPAD);
+      int i = 0;
+      for (; i < n_tiles; ++i) {
+        const int s = i % S::kStages;
+        const uint32_t ph = (i / S::kStages) & 1;
+        const int buf = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        if (!mbar_wait(acce_bar(buf), aph ^ 1, abort_flag)) { raise_abort(abort_flag, p.status); break; }
+        if (!mbar_wait(full_bar(s), ph, abort_flag)) { raise_abort(abort_flag, p.status); break; }
+        tc_fence_after();
+        const uint32_t a = smem_addr(stages + s * S::kStageBytes);
+        const uint32_t bq = a + S::kParts * S::kAPart;
+        const uint32_t d_tmem = tmem_base + buf * S::kAccStride;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int part = k >> 2;
+          const uint32_t off = (k & 3) * 32;   // 16 bf16 = 32 bytes along the swizzled row
+          tc_mma_bf16(d_tmem, smem_desc_sw128(a + part * S::kAPart + off),
+                      smem_desc_sw128(bq + part * S::kBPart + off), idesc, k > 0 ? 1u : 0u);
+        }
+        tc_commit(empty_bar(s));
+        tc_commit(accf_bar(buf));
+      }
+      if (i > 0) {   // all issued MMAs complete before TMEM is released
+        volatile int never = 0;
+        tc_commit(drain_bar);
+        mbar_wait(drain_bar, 0, &never);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;                  // TMEM lanes [32*quad, 32*quad + 32)
+    const uint64_t pol_z = policy_evict_last();
+    uint32_t rmin[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+    uint32_t rmax[2] = {0u, 0u};
+    int seg_b = -1, seg_kh = -1;
+    auto flush = [&]() {
+      if (seg_b >= 0 && p.stat_min != nullptr) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int h = lane + 32 * r;
+          if (h < p.g && rmin[r] <= rmax[r]) {
+            const int bj = seg_b * p.h_q + seg_kh * p.g + h;
+            atomicMin(p.stat_min + bj, rmin[r]);
+            atomicMax(p.stat_max + bj, rmax[r]);
+          }
+        }
+      }
+      rmin[0] = rmin[1] = 0xFFFFFFFFu;
+      rmax[0] = rmax[1] = 0u;
+    };
+    if (n_tiles > 0) {
+      TileCursor c;
+      c.seek(u0, unit_off, lens, p.B, p.h_k);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int buf = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        // every lane waits; the decision to go on is taken warp-uniformly
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(accf_bar(buf), aph, abort_flag));
+        if (!ok) { if (lane == 0) raise_abort(abort_flag, p.status); break; }
+        tc_fence_after();
+        float acc[NPAD];
+#pragma unroll
+        for (int cc = 0; cc < NPAD / 16; ++cc) {
+          float v[16];
+          tmem_ld_16(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * S::kAccStride + cc * 16, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[cc * 16 + e] = v[e];
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acce_bar(buf));
+
+        if (c.b != seg_b || c.kh != seg_kh) { flush(); seg_b = c.b; seg_kh = c.kh; }
+        const int pos = c.t * kTileM + quad * 32 + lane;
+        const bool valid = pos < c.Lb;
+        float* zrow = p.z + static_cast<long long>(c.b * p.h_q + c.kh * p.g) * p.z_stride + pos;
+#pragma unroll
+        for (int h = 0; h < NPAD; ++h) {
+          if (h < p.g) {
+            // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
+            const float zz = __fadd_rn(__fmul_rn(acc[h], p.scale), 0.0f);
+            if (valid) st_global_hint(zrow + h * p.z_stride, zz, pol_z);
+            const uint32_t key = ordered_key(zz);
+            const uint32_t kmin = __reduce_min_sync(0xffffffffu, valid ? key : 0xFFFFFFFFu);
+            const uint32_t kmax = __reduce_max_sync(0xffffffffu, valid ? key : 0u);
+            if (lane == (h & 31)) {
+              rmin[h >> 5] = min(rmin[h >> 5], kmin);
+              rmax[h >> 5] = max(rmax[h >> 5], kmax);
+            }
+          }
+        }
+        c.next(unit_off, lens, p.B, p.h_k);
+      }
+      flush();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+}  // namespace saga
