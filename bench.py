@@ -1,0 +1,433 @@
+#!/usr/bin/env python3
+"""Throughput of SAGA + Atop-N decode attention on B200.
+
+One step = one decode token of a batch of 16 sequences through 28 layers of
+Qwen2.5-1.5B-shaped SAGA attention at 32K context: h_q = 12, h_k = 1, h_v = 2,
+d = 128, N = 1024, i.e. 28 calls of the library's decode step on 28 distinct
+synthetic KV caches (11.3 GB, far above L2, so no L2 flush is needed).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl saga|reference]
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload (replicas:
+the decode step needs no exchange between GPUs); the timed region is bracketed
+by a barrier and a device synchronize, and the time is the maximum over ranks.
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (the
+plain float64 restatement of the method) on a bounded sample of the same
+workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "decode-attn tokens/sec and achieved HBM GB/s (% of B200 roofline) at 32K ctx"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "score_kernel_qwen32k.md")
+SCORE_SOURCES = [os.path.join(ROOT, "sparse_asymmetric_gqa_b200", "csrc", f)
+                 for f in ("score_kernel.cuh", "ptx.cuh")]
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["saga", "reference"], default="saga")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU work budget of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Maximum of a per-rank float over all ranks (no-op for one rank)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def score_source_hash():
+    h = hashlib.sha256()
+    for p in SCORE_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per score-kernel launch from the committed ncu summary, or
+    None if the kernel source changed since it was captured."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != score_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms in the background."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if uuid:
+            cmd += ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for t, s in self.samples if t0 <= t <= t1] or [s for _, s in self.samples]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in next(csv.reader(io.StringIO(r)))]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle leg
+
+def oracle_sample(spec, q, k, v, lens, budget_s):
+    """Time the CPU oracle on batch rows 0, 1, ... of one layer (all heads)
+    until about budget_s seconds of work; returns (rows, seconds, threads)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    rows, spent = 0, 0.0
+    while rows < q.shape[0] and (rows == 0 or spent < budget_s):
+        b = rows
+        qb = q[b:b + 1].float().cpu().numpy()
+        kb = k[b:b + 1].float().cpu().numpy()
+        vb = v[b:b + 1].float().cpu().numpy()
+        lb = np.array([int(lens[b])])
+        t0 = time.perf_counter()
+        oracle.decode_attn(qb, kb, vb, lb, spec.h_q, spec.h_k, spec.h_v, spec.N)
+        spent += time.perf_counter() - t0
+        rows += 1
+    return rows, spent, threads
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is one batch row of one layer."""
+    from sparse_asymmetric_gqa_b200 import workload
+    if rank != 0:
+        return
+    spec = workload.QWEN_32K
+    small = workload.scaled(spec, batch=2)
+    inp = workload.make_inputs(small)          # the first two rows' recipe, drawn on the CPU
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    q, k, v = (t.float().numpy() for t in (inp.q, inp.k_cache, inp.v_cache))
+    lens = inp.seq_lens.numpy()
+
+    def step(i):
+        b = i % small.batch
+        oracle.decode_attn(q[b:b + 1], k[b:b + 1], v[b:b + 1], lens[b:b + 1],
+                           spec.h_q, spec.h_k, spec.h_v, spec.N)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    # one step = one sequence through one layer; a token needs 28 layers
+    tok_s = args.steps / (dt * spec.layers)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "batch": spec.batch, "seq_len": spec.seq_len,
+                   "layers_per_token": spec.layers, "h_q": spec.h_q, "h_k": spec.h_k,
+                   "h_v": spec.h_v, "head_dim": spec.head_dim, "N": spec.N,
+                   "step": "one sequence through one layer (CPU float64 oracle)"},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{args.steps} (sequence, layer) calls of the Qwen-shaped "
+                                   "32K workload, first two batch rows of layer 0"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- CUDA leg
+
+def run_saga(args, rank, world, local):
+    from sparse_asymmetric_gqa_b200 import SagaDecoder, workload
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    spec = workload.QWEN_32K
+    L = spec.layers
+    B = spec.batch
+
+    layers = [workload.make_inputs(spec, layer=l, device=dev, seed=spec.seed + l + 100 * rank)
+              for l in range(L)]
+    outs = [torch.empty(B, spec.h_q, spec.head_dim, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    dec = SagaDecoder(B, spec.seq_len, spec.h_q, spec.h_k, spec.h_v, spec.head_dim, spec.N, device=dev)
+
+    def step():
+        for x, o in zip(layers, outs):
+            dec.attn(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=o)
+
+    # eager warm-up (also validates), then one CUDA graph per step
+    step()
+    status = dec.status()
+    if status & 0xFF:
+        raise RuntimeError(f"device status 0x{status:x}")
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    dec.profile(True, L)
+    n0 = dec.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    launches_per_step = dec.launch_count() - n0
+
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    time.sleep(0.5 if clocks else 0)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, world)
+    # per-kernel times of the last replay inside the timed region
+    score_ms, call_ms, n_prof = dec.profile_read()
+    dec.profile(False)
+
+    # ---- end to end through the host-buffer entry point (q in, out back, per layer)
+    pin_q = [x.q.cpu().pin_memory() for x in layers]
+    pin_l = [x.seq_lens.cpu().pin_memory() for x in layers]
+    pin_o = [torch.empty(B, spec.h_q, spec.head_dim, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+
+    def step_host():
+        for x, qh, lh, oh in zip(layers, pin_q, pin_l, pin_o):
+            dec.attn_host(qh, x.k_cache, x.v_cache, lh, spec.N, oh)
+
+    for _ in range(3):
+        step_host()
+    torch.cuda.synchronize(dev)
+    e_steps = max(1, min(args.steps, 50))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record()
+    for _ in range(e_steps):
+        step_host()
+        torch.cuda.current_stream(dev).synchronize()      # the step's result is on the host
+    h1.record()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1), world)
+    if not torch.equal(pin_o[0], outs[0].cpu()):
+        raise RuntimeError("host entry point result differs from the device call")
+    if clocks:
+        clocks.stop()
+
+    if rank != 0:
+        return
+    # ---- numbers
+    lens = [int(x) for x in layers[0].seq_lens.tolist()]
+    k_bytes = sum(spec.h_k * Lb * spec.head_dim * 2 for Lb in lens)           # per call
+    v_bytes_model = sum(spec.h_v * min(spec.N, Lb) * spec.head_dim * 2 for Lb in lens)
+    v_bytes_per_head = sum(spec.h_q * min(spec.N, Lb) * spec.head_dim * 2 for Lb in lens)
+    model_bytes = k_bytes + v_bytes_model
+    peak, peak_src = measured_hbm_peak()
+    step_s = ms_max / 1e3 / args.steps
+    value = world * B / step_s
+    score_avg_s = score_ms / 1e3 / max(n_prof, 1)
+    call_avg_s = call_ms / 1e3 / max(n_prof, 1)
+    achieved = k_bytes / score_avg_s / 1e9
+    call_gbs = model_bytes / call_avg_s / 1e9
+    traffic = profiled_traffic()
+    e2e_step_s = e2e_ms / 1e3 / e_steps
+    rows, spent, threads = oracle_sample(spec, layers[0].q, layers[0].k_cache, layers[0].v_cache,
+                                         lens, args.cpu_seconds)
+    cpu_tok_s = rows / (spent * L)
+    csum = clocks.summary(t_wall0, t_wall1) if clocks else {}
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": spec.name, "batch": B, "seq_len": spec.seq_len, "layers_per_step": L,
+            "h_q": spec.h_q, "h_k": spec.h_k, "h_v": spec.h_v, "head_dim": spec.head_dim,
+            "N": spec.N, "planted_keys": "2% per key head, s ~ U[2,4]",
+            "accumulate": "fp32", "timing": "CUDA graph of one step, K replays, CUDA events",
+            "l2": "no flush: each step reads 28 distinct caches (11.3 GB) >> 126 MB L2",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "kernel": "score_kernel (S1, q.K over the whole key cache)",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": traffic,
+            "algorithmic_bytes_per_launch": k_bytes, "avg_launch_us": score_avg_s * 1e6,
+            "peak_source": peak_src,
+        },
+        "call_roofline": {
+            "model_bytes_per_call": model_bytes, "avg_call_us": call_avg_s * 1e6,
+            "achieved": call_gbs, "frac": call_gbs / peak, "unit": "GB/s",
+            "model": "K cache over valid positions + N V rows per value head",
+            "v_bytes_per_query_head_model": v_bytes_per_head,
+        },
+        "cpu_baseline": {
+            "value": cpu_tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} batch rows x 12 heads of layer 0 ({spent:.1f} s of CPU work), "
+                      "scaled by 28 layers per token",
+        },
+        "e2e": {
+            "value": world * B / e2e_step_s, "unit": "tokens/s",
+            "h2d_bytes_per_step": L * (pin_q[0].numel() * 2 + pin_l[0].numel() * 4),
+            "d2h_bytes_per_step": L * pin_o[0].numel() * 2,
+            "path": "saga_decode_attn_host per layer (pinned q/seq_lens in, out back), "
+                    "eager, one host sync per step",
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": csum,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_saga(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -78,6 +78,8 @@ extern "C" {
 #define SAGA_STATUS_BAD_INDEX     0x4   /* saga_combine got an index >= L_b: that slot ignored */
 #define SAGA_STATUS_INFO_EXACT_FALLBACK 0x100  /* informational: a row needed the full radix
                                                    select (very flat score rows); not an error */
+#define SAGA_STATUS_INFO_ROBUST_PATH 0x200     /* informational: a row's sampled threshold bound
+                                                   missed and the histogram path ran; not an error */
 
 typedef struct saga_ctx* saga_handle;
 
@@ -86,7 +88,8 @@ typedef struct saga_ctx* saga_handle;
  * head_dim, and selections of up to max_N positions.  cuda_stream is a
  * cudaStream_t (NULL = legacy default stream).  The current CUDA device at
  * this call is the handle's device.  Workspace: about
- * 4*max_batch*h_q*(round_up(max_seq_len,32) + 2*max_N + 2) bytes.
+ * 4*max_batch*h_q*(round_up(max_seq_len,32) + 2*max_N + 3 +
+ * ceil(min(max_N,max_seq_len)/256)*(head_dim+2)) bytes.
  * Returns SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_CUDA. */
 SAGA_API int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len,
                      int h_q, int h_k, int h_v, int head_dim, int max_N,
@@ -139,10 +142,11 @@ SAGA_API int saga_select(saga_handle h, const float* scores, int scores_stride,
                 const int32_t* seq_lens, int h_q, int N,
                 int32_t* sel_idx, float* sel_logit);
 
-/* Stages S3+S4 alone ([MVK] Eq. (7)): softmax over the valid entries of each
- * selection row ([B][h_q][N]; entries with sel_idx < 0 are padding, entries
- * >= L_b are ignored and flagged SAGA_STATUS_BAD_INDEX) and the gathered P.V
- * over v_cache, bf16 out.  A row with no valid entry gets zeros. */
+/* Stages S3+S4 alone ([MVK] Eq. (7)): softmax over the valid entries among
+ * the first min(N, L_b) slots of each selection row ([B][h_q][N]; entries
+ * with sel_idx < 0 are padding, entries >= L_b are ignored and flagged
+ * SAGA_STATUS_BAD_INDEX) and the gathered P.V over v_cache, bf16 out.  A row
+ * with no valid entry gets zeros.  1 <= N <= max_N. */
 SAGA_API int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
                  const void* v_cache, const int32_t* seq_lens, int h_q, int h_v,
                  int head_dim, int N, void* out);
@@ -158,8 +162,10 @@ SAGA_API int saga_decode_launch_count(saga_handle h, long long* count);
 
 /* Profiling: when enabled, each decode call records CUDA events around its
  * score kernel and around the whole call on the handle's stream (up to
- * max_calls calls).  saga_decode_profile_read synchronises and returns the
- * summed milliseconds and the number of calls recorded, then resets. */
+ * max_calls calls; inside CUDA-graph capture the records become graph nodes,
+ * so every replay re-records them).  saga_decode_profile_read synchronises and
+ * returns the summed milliseconds and the number of calls recorded, then
+ * starts counting calls from zero again. */
 SAGA_API int saga_decode_profile(saga_handle h, int enable, int max_calls);
 SAGA_API int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms,
                              int* n_calls);

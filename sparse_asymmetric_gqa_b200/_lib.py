@@ -14,6 +14,7 @@ SAGA_STATUS_BAD_SEQ_LEN = 0x1
 SAGA_STATUS_TIMEOUT = 0x2
 SAGA_STATUS_BAD_INDEX = 0x4
 SAGA_STATUS_INFO_EXACT_FALLBACK = 0x100
+SAGA_STATUS_INFO_ROBUST_PATH = 0x200
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int

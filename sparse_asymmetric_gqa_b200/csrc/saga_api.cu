@@ -1,9 +1,10 @@
 // saga_api.cu -- the C ABI declared in include/saga.h: argument validation,
 // the handle and its workspace, TMA descriptor encoding and the launch plan.
 //
-// One decode call enqueues two kernels on the handle's stream:
-//   score_kernel          S1, persistent, one CTA per SM (tcgen05 + TMA)
-//   select_combine_kernel S2-S4, one CTA per (batch row, query head)
+// One decode call enqueues three kernels on the handle's stream:
+//   score_kernel   S1, persistent, one CTA per SM (tcgen05 + TMA)
+//   select_kernel  S2, one CTA per (batch row, query head)
+//   gather_kernel  S3 + S4, one CTA per 256 selected rows of a (b, j)
 // Nothing is allocated, synchronised or copied to the host on that path.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -21,6 +22,7 @@
 #include "ptx.cuh"
 #include "score_kernel.cuh"
 #include "select_kernel.cuh"
+#include "gather_kernel.cuh"
 
 using namespace saga;
 
@@ -81,6 +83,9 @@ struct saga_ctx {
   __nv_bfloat16* q_stage = nullptr;
   __nv_bfloat16* out_stage = nullptr;
   int32_t* lens_stage = nullptr;
+  float* partial = nullptr;       // gather partials [rows][max_chunks][d + 2]
+  uint32_t* counter = nullptr;    // gather merge counters [rows]
+  int max_chunks = 0;
   long long launches = 0;
   // profiling
   bool prof = false;
@@ -103,16 +108,7 @@ int set_smem_attrs_once() {
     SAGA_ATTR(128, 16) SAGA_ATTR(128, 32) SAGA_ATTR(128, 48) SAGA_ATTR(128, 64)
 #undef SAGA_ATTR
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(select_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sizeof(SelectSmem)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(select_combine_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sizeof(SelectSmem)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sizeof(SelectSmem)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(combine_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sizeof(SelectSmem)));
     rc = (e == cudaSuccess) ? 0 : 1;
   });
@@ -161,13 +157,13 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
 }
 
 int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
-                  const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_logit,
-                  const void* v_cache, void* out) {
+                  const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_logit) {
   SelectParams p;
   p.z = z;
   p.z_stride = z_stride;
   p.stat_min = stats ? h->stat_min : nullptr;
   p.stat_max = stats ? h->stat_max : nullptr;
+  p.gather_count = h->counter;
   p.seq_lens = seq_lens;
   p.B = h->batch;
   p.h_q = h->h_q;
@@ -176,17 +172,36 @@ int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
   p.z_vec4 = ((z_stride % 4) == 0 && (reinterpret_cast<uintptr_t>(z) % 16) == 0) ? 1 : 0;
   p.sel_idx = sel_idx;
   p.sel_logit = sel_logit;
+  p.status = h->status;
+  select_kernel<<<h->batch * h->h_q, kSelThreads, sizeof(SelectSmem), h->stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+  ++h->launches;
+  return SAGA_OK;
+}
+
+int launch_gather(saga_ctx* h, const int32_t* sel_idx, const float* sel_logit,
+                  const int32_t* seq_lens, const void* v_cache, int N, void* out) {
+  GatherParams p;
+  p.sel_idx = sel_idx;
+  p.sel_logit = sel_logit;
+  p.seq_lens = seq_lens;
   p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.h_q = h->h_q;
   p.h_v = h->h_v;
   p.g_v = h->g_v;
+  p.L_max = h->max_seq_len;
+  p.N = N;
+  p.partial = h->partial;
+  p.max_chunks = h->max_chunks;
+  p.counter = h->counter;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = h->status;
-  const int grid = h->batch * h->h_q;
-  const size_t smem = sizeof(SelectSmem);
+  const int slots = N < h->max_seq_len ? N : h->max_seq_len;
+  const dim3 grid(h->batch * h->h_q, (slots + kGatherRows - 1) / kGatherRows);
   if (h->d == 64)
-    select_combine_kernel<64><<<grid, kSelThreads, smem, h->stream>>>(p);
+    gather_kernel<64><<<grid, kGatherThreads, 0, h->stream>>>(p);
   else
-    select_combine_kernel<128><<<grid, kSelThreads, smem, h->stream>>>(p);
+    gather_kernel<128><<<grid, kGatherThreads, 0, h->stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
   ++h->launches;
   return SAGA_OK;
@@ -195,6 +210,15 @@ int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
 int check_heads(saga_ctx* h, int h_q, int h_k, int h_v, int d) {
   if (h_q != h->h_q || h_k != h->h_k || h_v != h->h_v || d != h->d) return SAGA_ERR_INVALID_ARG;
   return SAGA_OK;
+}
+
+// Inside stream capture an event record becomes a graph node only with the
+// external flag; then each replay re-records it and elapsed times stay valid.
+cudaError_t record_event(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  return cudaEventRecord(e, s);
 }
 
 struct DeviceGuard {   // run a call on the handle's device, restore the caller's
@@ -218,18 +242,20 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   if (!dg.ok) return SAGA_ERR_CUDA;
   const bool prof = h->prof && h->prof_n < h->prof_max;
   cudaEvent_t* ev = prof ? &h->ev[3 * h->prof_n] : nullptr;
-  if (prof && cudaEventRecord(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (prof && record_event(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
   int rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true);
   if (rc) return rc;
-  if (prof && cudaEventRecord(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
   // The selection goes to the caller's arrays when given, else to the workspace
   // (row stride N either way).
   int32_t* si = sel_idx ? sel_idx : h->sel_idx;
   float* sl = sel_logit ? sel_logit : h->sel_logit;
-  rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl, v_cache, out);
+  rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl);
+  if (rc) return rc;
+  rc = launch_gather(h, si, sl, seq_lens, v_cache, N, out);
   if (rc) return rc;
   if (prof) {
-    if (cudaEventRecord(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     ++h->prof_n;
   }
   return SAGA_OK;
@@ -289,9 +315,13 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   const size_t stat_bytes = rows * sizeof(uint32_t);
   const size_t sel_bytes = rows * static_cast<size_t>(max_N) * 4;
   const size_t qo_bytes = rows * head_dim * 2;
+  const int slots = max_N < max_seq_len ? max_N : max_seq_len;
+  h->max_chunks = (slots + kGatherRows - 1) / kGatherRows;
+  const size_t part_bytes = rows * h->max_chunks * (head_dim + 2) * sizeof(float);
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t total = al(z_bytes) + 2 * al(stat_bytes) + 2 * al(sel_bytes) + al(256) +
-                       2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4);
+                       2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4) +
+                       al(part_bytes) + al(stat_bytes);
   if (cudaMalloc(&h->ws, total) != cudaSuccess) { delete h; return SAGA_ERR_CUDA; }
   uint8_t* w = static_cast<uint8_t*>(h->ws);
   h->z = reinterpret_cast<float*>(w); w += al(z_bytes);
@@ -302,8 +332,11 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->status = reinterpret_cast<int*>(w); w += al(256);
   h->q_stage = reinterpret_cast<__nv_bfloat16*>(w); w += al(qo_bytes);
   h->out_stage = reinterpret_cast<__nv_bfloat16*>(w); w += al(qo_bytes);
-  h->lens_stage = reinterpret_cast<int32_t*>(w);
+  h->lens_stage = reinterpret_cast<int32_t*>(w); w += al(static_cast<size_t>(max_batch) * 4);
+  h->partial = reinterpret_cast<float*>(w); w += al(part_bytes);
+  h->counter = reinterpret_cast<uint32_t*>(w);
   if (cudaMemset(h->stat_min, 0xFF, stat_bytes) != cudaSuccess ||
+      cudaMemset(h->counter, 0x00, stat_bytes) != cudaSuccess ||
       cudaMemset(h->stat_max, 0x00, stat_bytes) != cudaSuccess ||
       cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->ws);
@@ -382,8 +415,7 @@ int saga_select(saga_handle h, const float* scores, int scores_stride, const int
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
-  return launch_select(h, scores, scores_stride, false, seq_lens, N, sel_idx, sel_logit,
-                       nullptr, nullptr);
+  return launch_select(h, scores, scores_stride, false, seq_lens, N, sel_idx, sel_logit);
 }
 
 int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
@@ -391,32 +423,14 @@ int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
                  int N, void* out) {
   if (!h || !sel_idx || !sel_logit || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
   if (h_q != h->h_q || h_v != h->h_v || head_dim != h->d) return SAGA_ERR_INVALID_ARG;
-  if (N < 1) return SAGA_ERR_INVALID_ARG;
+  if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
-  SelectParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.seq_lens = seq_lens;
-  p.B = h->batch;
-  p.h_q = h->h_q;
-  p.L_max = h->max_seq_len;
-  p.N = N;
-  p.sel_idx = const_cast<int32_t*>(sel_idx);
-  p.sel_logit = const_cast<float*>(sel_logit);
-  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
-  p.h_v = h->h_v;
-  p.g_v = h->g_v;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.status = h->status;
-  const int grid = h->batch * h->h_q;
-  const size_t smem = sizeof(SelectSmem);
-  if (h->d == 64)
-    combine_kernel<64><<<grid, kSelThreads, smem, h->stream>>>(p);
-  else
-    combine_kernel<128><<<grid, kSelThreads, smem, h->stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
-  ++h->launches;
-  return SAGA_OK;
+  // no select kernel ran before: clear the merge counters here
+  if (cudaMemsetAsync(h->counter, 0, static_cast<size_t>(h->batch) * h->h_q * sizeof(uint32_t),
+                      h->stream) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+  return launch_gather(h, sel_idx, sel_logit, seq_lens, v_cache, N, out);
 }
 
 int saga_decode_status(saga_handle h, int* device_status) {

@@ -14,9 +14,10 @@
 //     memory stages with TMA (128-byte swizzle, L2 evict-first for K);
 //   * warp 1 issues tcgen05.mma (M = 128 positions, N = g padded to 16k,
 //     K = 16 per instruction) into a double-buffered TMEM accumulator;
-//   * warps 2-5 read the accumulator back with tcgen05.ld (thread = position,
-//     registers = heads), scale, store z row-wise (coalesced per head) and keep
-//     per-(b, j) min/max statistics for the selector's first pass.
+//   * warps 2-9 read the accumulator back with tcgen05.ld (thread = position,
+//     registers = heads; two warps per TMEM lane quarter, each taking half of
+//     the heads), scale, store z row-wise (coalesced per head) and keep
+//     per-(b, j) min/max statistics in registers for the selector.
 #pragma once
 
 #include <cuda.h>
@@ -25,7 +26,8 @@
 namespace saga {
 
 constexpr int kTileM = 128;          // positions per tile (MMA M)
-constexpr int kScoreThreads = 192;   // 6 warps: TMA, MMA, 4 x epilogue
+constexpr int kScoreThreads = 320;   // 10 warps: TMA, MMA, 8 x epilogue
+constexpr int kEpiWarps = 8;
 constexpr int kMaxBatch = 1024;
 
 struct ScoreParams {
@@ -122,7 +124,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
   if (warp == 0) {
     if (lane == 0) {
       for (int s = 0; s < S::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-      for (int i = 0; i < 2; ++i) { mbar_init(accf_bar(i), 1); mbar_init(acce_bar(i), 4); }
+      for (int i = 0; i < 2; ++i) { mbar_init(accf_bar(i), 1); mbar_init(acce_bar(i), kEpiWarps); }
       mbar_init(drain_bar, 1);
       *abort_flag = 0;
       fence_mbar_init();
@@ -230,25 +232,33 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;                  // TMEM lanes [32*quad, 32*quad + 32)
+    // Warp w reads TMEM lane quarter w % 4 (the hardware rule) and heads
+    // [half * H, half * H + H) of the group, half = (w - 2) / 4.
+    constexpr int H = NPAD / 2;
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int h0 = half * H;
     const uint64_t pol_z = policy_evict_last();
-    uint32_t rmin[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
-    uint32_t rmax[2] = {0u, 0u};
+    uint32_t rmin[H], rmax[H];
+#pragma unroll
+    for (int i = 0; i < H; ++i) { rmin[i] = 0xFFFFFFFFu; rmax[i] = 0u; }
     int seg_b = -1, seg_kh = -1;
     auto flush = [&]() {
-      if (seg_b >= 0 && p.stat_min != nullptr) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int h = lane + 32 * r;
-          if (h < p.g && rmin[r] <= rmax[r]) {
+      for (int i = 0; i < H; ++i) {
+        const int h = h0 + i;
+        if (h < p.g) {
+          const uint32_t kmin = __reduce_min_sync(0xffffffffu, rmin[i]);
+          const uint32_t kmax = __reduce_max_sync(0xffffffffu, rmax[i]);
+          if (lane == 0 && seg_b >= 0 && p.stat_min != nullptr && kmin <= kmax) {
             const int bj = seg_b * p.h_q + seg_kh * p.g + h;
-            atomicMin(p.stat_min + bj, rmin[r]);
-            atomicMax(p.stat_max + bj, rmax[r]);
+            atomicMin(p.stat_min + bj, kmin);
+            atomicMax(p.stat_max + bj, kmax);
           }
         }
+        rmin[i] = 0xFFFFFFFFu;
+        rmax[i] = 0u;
       }
-      rmin[0] = rmin[1] = 0xFFFFFFFFu;
-      rmax[0] = rmax[1] = 0u;
     };
     if (n_tiles > 0) {
       TileCursor c;
@@ -260,13 +270,14 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const bool ok = __all_sync(0xffffffffu, mbar_wait(accf_bar(buf), aph, abort_flag));
         if (!ok) { if (lane == 0) raise_abort(abort_flag, p.status); break; }
         tc_fence_after();
-        float acc[NPAD];
+        float acc[H];
 #pragma unroll
-        for (int cc = 0; cc < NPAD / 16; ++cc) {
-          float v[16];
-          tmem_ld_16(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * S::kAccStride + cc * 16, v);
+        for (int cc = 0; cc < H / 8; ++cc) {
+          float v[8];
+          tmem_ld_8(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * S::kAccStride +
+                        h0 + cc * 8, v);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) acc[cc * 16 + e] = v[e];
+          for (int e = 0; e < 8; ++e) acc[cc * 8 + e] = v[e];
         }
         tmem_wait_ld();
         tc_fence_before();
@@ -275,20 +286,17 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
         if (c.b != seg_b || c.kh != seg_kh) { flush(); seg_b = c.b; seg_kh = c.kh; }
         const int pos = c.t * kTileM + quad * 32 + lane;
-        const bool valid = pos < c.Lb;
-        float* zrow = p.z + static_cast<long long>(c.b * p.h_q + c.kh * p.g) * p.z_stride + pos;
+        if (pos < c.Lb) {
+          float* zrow = p.z + static_cast<long long>(c.b * p.h_q + c.kh * p.g + h0) * p.z_stride + pos;
 #pragma unroll
-        for (int h = 0; h < NPAD; ++h) {
-          if (h < p.g) {
-            // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
-            const float zz = __fadd_rn(__fmul_rn(acc[h], p.scale), 0.0f);
-            if (valid) st_global_hint(zrow + h * p.z_stride, zz, pol_z);
-            const uint32_t key = ordered_key(zz);
-            const uint32_t kmin = __reduce_min_sync(0xffffffffu, valid ? key : 0xFFFFFFFFu);
-            const uint32_t kmax = __reduce_max_sync(0xffffffffu, valid ? key : 0u);
-            if (lane == (h & 31)) {
-              rmin[h >> 5] = min(rmin[h >> 5], kmin);
-              rmax[h >> 5] = max(rmax[h >> 5], kmax);
+          for (int e = 0; e < H; ++e) {
+            if (h0 + e < p.g) {
+              // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
+              const float zz = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
+              st_global_hint(zrow + e * p.z_stride, zz, pol_z);
+              const uint32_t key = ordered_key(zz);
+              rmin[e] = min(rmin[e], key);
+              rmax[e] = max(rmax[e], key);
             }
           }
         }

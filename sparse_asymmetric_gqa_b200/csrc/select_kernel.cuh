@@ -1,30 +1,38 @@
-// select_kernel.cuh -- S2 (exact top-N selection), S3 (softmax over the
-// selection) and S4 (gathered P.V) for one (batch row b, query head j) per CTA.
+// select_kernel.cuh -- S2, exact top-N selection of each (batch row b, query
+// head j) score row, one CTA per row.
 //
-// Selection ("More Value per Key", §2.5 Eq. (6); Atop-N, §3.1 and App. C.1):
-// Atop-N finds the N-th largest score and keeps every score above it by a
-// plain per-element compare.  Here the threshold is found exactly on every
-// call, in three passes over the fp32 score row (which the score pass left in
-// L2):
-//   A  histogram of the row over 2048 equal-width bins between the row's min
-//      and max (the score pass supplies both), which spreads N(0,1)-like rows
-//      evenly over the bins, so shared-memory atomics rarely collide;
-//   B  gather the keys of the one bin that holds the N-th score (typically a
-//      few dozen) and radix-select inside it (4 x 8-bit digits on
-//      order-preserving uint32 keys) -> exact threshold key T and the number of
-//      ties at T still needed;
-//   C  compare pass in position order with a block-wide scan: keep z > T and
-//      the lowest-index ties = T, writing positions ascending.
-// Binning is monotone in z (a rounded subtract, a rounded multiply by a
-// non-negative scale, clamp, truncate), so a higher bin always means a
-// strictly larger score; any min/max (even a stale or missing one) gives a
-// correct result.  If the boundary bin overflows the candidate buffer (very
-// flat rows) the radix select runs over the whole row instead.
-//
-// Softmax and P.V ("More Value per Key", §3.1 Eq. (7)): weights exp(z - m)
-// with m the largest selected score, fp32 accumulation of the gathered value
-// rows (one warp per row, a lane per 2-4 elements), one bf16 rounding at the
-// end.
+// Atop-N ("More Value per Key", §3.1 and App. C.1) keeps every score at or
+// above a threshold by a plain per-element compare into a fixed-capacity
+// buffer, the threshold being the N-th largest score; top-N itself is §2.5
+// Eq. (6).  Here the threshold is exact and found on every call:
+//   1  the row is streamed into shared memory by 1-D TMA bulk copies (a ring of
+//      kRing x 16 KB, started at kernel entry);
+//   2  meanwhile a lower bound t_lo for the N-th score comes from an evenly
+//      spread sample of the row (up to 128 blocks of 32 scores): an
+//      equal-width histogram of the sample and the lower edge of the bin below
+//      the one holding its (r_s + 6 sqrt(r_s) + 8)-th largest value,
+//      r_s = N * sample / L;
+//   3  one compare pass (z >= t_lo) appends (key, position) of every passing
+//      score to a candidate buffer of kCandCap entries;
+//   4  the exact N-th key T among the candidates (equal-width histogram between
+//      their min and max, the keys of the bin that holds the N-th, a one-warp
+//      rank count or a radix select inside it);
+//   5  the kept positions (key > T, and the lowest-position ties = T) are
+//      marked in a bitmap of the row; a scan of the bitmap's word popcounts
+//      gives each kept candidate its output slot, so positions come out
+//      ascending without a sort.
+// The result is exact whatever the sample says: if fewer than N_b scores pass
+// t_lo, more than kCandCap do, or the row is longer than the bitmap, the
+// robust path runs instead (histogram of the whole row over 2048 equal-width
+// bins between its min and max, the keys of the boundary bin, a radix select
+// inside it, one ordered compare pass).  The binning is monotone in z (a
+// rounded subtract, a rounded multiply by a non-negative scale, clamp,
+// truncate), so a higher bin always means a strictly larger score, for any
+// min/max.  Very flat rows whose boundary bin overflows fall back to a radix
+// select over the whole row.
+// Keys are order-preserving uint32 images of the fp32 scores, -0 folded onto
+// +0; ties at the N-th score go to the lowest position.  NaN scores are not
+// supported.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -35,37 +43,51 @@ namespace saga {
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kCandCap = 4096;
-constexpr int kItems = 8;                       // positions per thread per compaction chunk
-constexpr int kChunk = kSelThreads * kItems;    // 4096
+constexpr int kCandCap = 4096;                  // candidate buffer (key, position)
+constexpr int kBinKeys = 1024;                  // boundary-bin / tie scratch
+constexpr int kSampleBlocks = 128;              // sample: up to 128 blocks of 32 scores
+constexpr int kItems = 8;                       // scores per thread per chunk
+constexpr int kChunk = kSelThreads * kItems;    // 4096 scores = one 16 KB ring buffer
+constexpr int kRing = 3;                        // bulk-copy ring depth
+constexpr int kMaxBitmapL = 131072;             // longest row of the bitmap emission
 
 struct SelectParams {
   const float* z;               // [B*h_q][z_stride]
   long long z_stride;
   uint32_t* stat_min;           // ordered-key min/max per row, or nullptr
   uint32_t* stat_max;
+  uint32_t* gather_count;       // per-row counters of the gather kernel (reset here), or nullptr
   const int32_t* seq_lens;
   int B, h_q, L_max, N;
-  int z_vec4;                   // rows are 16-byte aligned
+  int z_vec4;                   // rows are 16-byte aligned (bulk copies allowed)
   int32_t* sel_idx;             // [B*h_q][N]
   float* sel_logit;
-  // S3 + S4 (skipped when out == nullptr)
-  const __nv_bfloat16* v_cache; // [B][h_v][L_max][D]
-  int h_v, g_v;
-  __nv_bfloat16* out;           // [B*h_q][D]
   int* status;
 };
 
 struct SelectSmem {
-  uint32_t hist[kBins];
   union {
-    uint32_t cand[kCandCap];
-    float red[kSelWarps][128];
-  } u;
+    float ring[kRing][kChunk];                  // compare-pass staging
+    struct {
+      uint32_t bits[kMaxBitmapL / 32];          // kept positions
+      uint32_t wpre[kMaxBitmapL / 32];          // exclusive popcount prefix per word
+    } bm;
+  } a;
+  union {
+    uint32_t sample[kSampleBlocks * 32];
+    struct {
+      uint32_t key[kCandCap];
+      int32_t pos[kCandCap];
+    } c;
+  } b;
+  uint32_t hist[kBins];
+  uint32_t bin_keys[kBinKeys];
+  uint64_t full[kRing];
+  uint32_t red[2 * kSelWarps];
   uint32_t scan[kSelWarps];
   uint32_t bcast[4];
-  float fred[kSelWarps];
   uint32_t cand_n;
+  uint32_t tie_n;
 };
 
 // Canonical key of a score: -0 is folded onto +0 first.
@@ -104,50 +126,32 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* scan, 
   return before + x - v;
 }
 
-__device__ __forceinline__ float block_max(float v, float* fred) {
-  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) fred[threadIdx.x >> 5] = v;
+// Block-wide min and max in one barrier round.
+__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, SelectSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) { sm.red[warp] = lo; sm.red[kSelWarps + warp] = hi; }
   __syncthreads();
-  float r = fred[0];
-  for (int w = 1; w < kSelWarps; ++w) r = fmaxf(r, fred[w]);
+  lo = sm.red[0];
+  hi = sm.red[kSelWarps];
+#pragma unroll
+  for (int w = 1; w < kSelWarps; ++w) { lo = min(lo, sm.red[w]); hi = max(hi, sm.red[kSelWarps + w]); }
   __syncthreads();
-  return r;
 }
 
-__device__ __forceinline__ uint32_t block_min_u32(uint32_t v, uint32_t* scan) {
-  v = __reduce_min_sync(0xffffffffu, v);
-  if ((threadIdx.x & 31) == 0) scan[threadIdx.x >> 5] = v;
-  __syncthreads();
-  uint32_t r = scan[0];
-  for (int w = 1; w < kSelWarps; ++w) r = min(r, scan[w]);
-  __syncthreads();
-  return r;
-}
-
-__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* scan) {
-  v = __reduce_max_sync(0xffffffffu, v);
-  if ((threadIdx.x & 31) == 0) scan[threadIdx.x >> 5] = v;
-  __syncthreads();
-  uint32_t r = scan[0];
-  for (int w = 1; w < kSelWarps; ++w) r = max(r, scan[w]);
-  __syncthreads();
-  return r;
-}
-
-// MSB-first radix select: the k-th largest key among key(i), i < count (keys
-// outside the running prefix are skipped).  Returns the key T and, in *need,
-// how many elements equal to T belong to the top k (k - #(key > T)).
-template <class KeyAt>
-__device__ uint32_t radix_select(KeyAt key_at, int count, uint32_t k, SelectSmem& sm,
-                                 uint32_t* need) {
+// MSB-first radix select over a key set: visit(f) makes every thread call
+// f(key) for its own share of the set.  Returns the k-th largest key T and,
+// in *need, how many keys equal to T belong to the top k (k - #(key > T)).
+template <class Visit>
+__device__ uint32_t radix_select(Visit visit, uint32_t k, SelectSmem& sm, uint32_t* need) {
   uint32_t prefix = 0, mask = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += kSelThreads) sm.hist[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < count; i += kSelThreads) {
-      const uint32_t key = key_at(i);
+    visit([&](uint32_t key) {
       if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
-    }
+    });
     __syncthreads();
     if (threadIdx.x < 32) {
       const int lane = threadIdx.x;
@@ -162,7 +166,7 @@ __device__ uint32_t radix_select(KeyAt key_at, int count, uint32_t k, SelectSmem
         const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      uint32_t above = incl - c;             // elements in higher digits
+      uint32_t above = incl - c;             // keys in higher digits
       for (int e = 7; e >= 0; --e) {
         const uint32_t h = sm.hist[d0 + e];
         if (above < k && above + h >= k) { sm.bcast[0] = d0 + e; sm.bcast[1] = above; }
@@ -180,115 +184,445 @@ __device__ uint32_t radix_select(KeyAt key_at, int count, uint32_t k, SelectSmem
   return prefix;
 }
 
-// S3 + S4 for one (b, j): weights exp(z - m) over the count selection slots
-// (slots with an index outside [0, L) carry no weight), fp32 accumulation of
-// the gathered value rows, one bf16 rounding.  Returns the number of slots
-// whose index was out of range.
-template <int D>
-__device__ int combine_rows(const SelectParams& p, int bj, const int32_t* idx_in,
-                            const float* logit_in, int count, int L, float m, SelectSmem& sm) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = bj / p.h_q, j = bj % p.h_q;
-  constexpr int EPL = D / 32;                     // elements per lane: 2 or 4
-  const __nv_bfloat16* vrow0 = p.v_cache +
-      (static_cast<long long>(b) * p.h_v + j / p.g_v) * p.L_max * D + lane * EPL;
-  float acc[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) acc[e] = 0.0f;
-  float s_local = 0.0f;
-  int bad = 0;
-  for (int r0 = warp * 32; r0 < count; r0 += kSelThreads) {
-    const int r = r0 + lane;
-    int my_idx = -1;
-    float my_w = 0.0f;
-    if (r < count) {
-      my_idx = idx_in[r];
-      if (my_idx >= L) { ++bad; my_idx = -1; }
-      if (my_idx >= 0) my_w = expf(logit_in[r] - m);
-    }
-    s_local += my_w;
-    const int cnt = min(32, count - r0);
-    for (int t0 = 0; t0 < cnt; t0 += 8) {
-      float wv[8];
-      uint2 raw4[8];
-      uint32_t raw2[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int id = __shfl_sync(0xffffffffu, my_idx, (t0 + u) & 31);
-        wv[u] = __shfl_sync(0xffffffffu, my_w, (t0 + u) & 31);
-        if (t0 + u < cnt && id >= 0) {
-          const __nv_bfloat16* src = vrow0 + static_cast<long long>(id) * D;
-          if constexpr (EPL == 4) raw4[u] = __ldg(reinterpret_cast<const uint2*>(src));
-          else raw2[u] = __ldg(reinterpret_cast<const uint32_t*>(src));
-        } else {
-          wv[u] = 0.0f;
-          if constexpr (EPL == 4) raw4[u] = make_uint2(0u, 0u);
-          else raw2[u] = 0u;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if constexpr (EPL == 4) {
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw4[u].x));
-          const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw4[u].y));
-          acc[0] = fmaf(wv[u], a.x, acc[0]);
-          acc[1] = fmaf(wv[u], a.y, acc[1]);
-          acc[2] = fmaf(wv[u], c2.x, acc[2]);
-          acc[3] = fmaf(wv[u], c2.y, acc[3]);
-        } else {
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw2[u]));
-          acc[0] = fmaf(wv[u], a.x, acc[0]);
-          acc[1] = fmaf(wv[u], a.y, acc[1]);
-        }
-      }
-    }
+// k-th largest of a set of at most 32 keys held one per lane of warp 0:
+// writes T to sm.bcast[0] and the ties needed to sm.bcast[1].
+__device__ __forceinline__ void warp_kth(uint32_t key, bool has, uint32_t k, SelectSmem& sm) {
+  uint32_t gt = 0, ge = 0;
+  for (int m = 0; m < 32; ++m) {
+    const uint32_t km = __shfl_sync(0xffffffffu, key, m);
+    const bool hm = __shfl_sync(0xffffffffu, has, m);
+    if (hm) { gt += km > key; ge += km >= key; }
   }
-  for (int o = 16; o; o >>= 1) s_local += __shfl_xor_sync(0xffffffffu, s_local, o);
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) sm.u.red[warp][lane * EPL + e] = acc[e];
-  if (lane == 0) sm.fred[warp] = s_local;
+  if (has && gt < k && k <= ge) { sm.bcast[0] = key; sm.bcast[1] = k - gt; }
+}
+
+// k-th largest key of a shared-memory key set (visit as in radix_select):
+// equal-width histogram between the set's min and max (rarely colliding
+// atomics), the keys of the bin holding the k-th, then an exact finish there.
+template <class Visit>
+__device__ uint32_t kth_largest(Visit visit, uint32_t k, SelectSmem& sm, uint32_t* need) {
+  const int tid = threadIdx.x;
+  uint32_t lo_k = 0xFFFFFFFFu, hi_k = 0u;
+  visit([&](uint32_t key) { lo_k = min(lo_k, key); hi_k = max(hi_k, key); });
+  block_minmax(lo_k, hi_k, sm);
+  if (lo_k == hi_k) { *need = k; return lo_k; }
+  const float lo = key_to_float(lo_k), hi = key_to_float(hi_k);
+  const float scale = static_cast<float>(kBins) / (hi - lo);
+  if (!(scale < INFINITY) || !(scale > 0.0f)) return radix_select(visit, k, sm, need);
+
+  for (int i = tid; i < kBins; i += kSelThreads) sm.hist[i] = 0;
+  if (tid == 0) sm.cand_n = 0;
   __syncthreads();
-  if (tid < D) {
-    float o = 0.0f, s = 0.0f;
-    for (int w2 = 0; w2 < kSelWarps; ++w2) { o += sm.u.red[w2][tid]; s += sm.fred[w2]; }
-    p.out[static_cast<long long>(bj) * D + tid] = __float2bfloat16_rn(s > 0.0f ? o / s : 0.0f);
+  visit([&](uint32_t key) { atomicAdd(&sm.hist[lin_bin(key_to_float(key), lo, scale)], 1u); });
+  __syncthreads();
+  {
+    const int b0 = 4 * (kSelThreads - 1 - tid);   // thread order runs over the bins top-down
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c += sm.hist[b0 + e];
+    uint32_t total;
+    uint32_t above = block_excl_scan(c, sm.scan, &total);
+    for (int e = 3; e >= 0; --e) {
+      const uint32_t h = sm.hist[b0 + e];
+      if (above < k && above + h >= k) { sm.bcast[0] = b0 + e; sm.bcast[1] = above; sm.bcast[2] = h; }
+      above += h;
+    }
   }
-  return bad;
+  __syncthreads();
+  const int bstar = static_cast<int>(sm.bcast[0]);
+  const uint32_t above = sm.bcast[1];
+  const uint32_t in_bin = sm.bcast[2];
+  const uint32_t k2 = k - above;
+  __syncthreads();
+  if (in_bin > static_cast<uint32_t>(kBinKeys)) return radix_select(visit, k, sm, need);
+  visit([&](uint32_t key) {
+    if (lin_bin(key_to_float(key), lo, scale) == bstar) sm.bin_keys[atomicAdd(&sm.cand_n, 1u)] = key;
+  });
+  __syncthreads();
+  if (in_bin <= 32) {
+    if (tid < 32) warp_kth(tid < static_cast<int>(in_bin) ? sm.bin_keys[tid] : 0u,
+                           tid < static_cast<int>(in_bin), k2, sm);
+    __syncthreads();
+    const uint32_t T = sm.bcast[0];
+    *need = sm.bcast[1];
+    __syncthreads();
+    return T;
+  }
+  return radix_select(
+      [&](auto f) {
+        for (int i = tid; i < static_cast<int>(in_bin); i += kSelThreads) f(sm.bin_keys[i]);
+      },
+      k2, sm, need);
 }
 
-// Stages S3 + S4 alone, from a caller-supplied selection (padding: index -1).
-template <int D>
-__global__ void __launch_bounds__(kSelThreads)
-combine_kernel(const SelectParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
-  const int bj = blockIdx.x;
-  const int b = bj / p.h_q;
-  const int L = p.seq_lens[b];
-  const int32_t* idx_in = p.sel_idx + static_cast<long long>(bj) * p.N;
-  const float* logit_in = p.sel_logit + static_cast<long long>(bj) * p.N;
-  if (L < 1 || L > p.L_max) {
-    if (threadIdx.x == 0) atomicOr(p.status, 0x1 /* SAGA_STATUS_BAD_SEQ_LEN */);
-    for (int e = threadIdx.x; e < D; e += kSelThreads)
-      p.out[static_cast<long long>(bj) * D + e] = __float2bfloat16_rn(0.0f);
-    return;
+// Eight consecutive scores starting at base; entries at or beyond `end` are
+// returned as -inf and masked by the caller.
+__device__ __forceinline__ void load8(const float* row, int base, int end, bool vec4, float (&v)[8]) {
+  if (vec4 && base + 7 < end) {
+    const float4 f0 = *reinterpret_cast<const float4*>(row + base);
+    const float4 f1 = *reinterpret_cast<const float4*>(row + base + 4);
+    v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+    v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (base + e < end) ? row[base + e] : -INFINITY;
   }
-  float m_local = -INFINITY;
-  for (int r = threadIdx.x; r < p.N; r += kSelThreads) {
-    const int id = idx_in[r];
-    if (id >= 0 && id < L) m_local = fmaxf(m_local, logit_in[r]);
-  }
-  const float m = block_max(m_local, sm.fred);
-  const int bad = combine_rows<D>(p, bj, idx_in, logit_in, p.N, L, m, sm);
-  if (bad) atomicOr(p.status, 0x4 /* SAGA_STATUS_BAD_INDEX */);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSelThreads)
-select_combine_kernel(const SelectParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+// Lower bound (a score value) for the n_b-th largest score of a row of
+// L > kChunk scores, from an evenly spread sample of blocks of 32 consecutive
+// scores.  Any value is safe: the caller counts what passes it.
+__device__ float sample_bound(const float* row, int L, int n_b, SelectSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nblk = min(kSampleBlocks, L / 32);
+  const int S = nblk * 32;
+  const int lpb = L / 32;                              // whole 32-score blocks in the row
+  float v[kSampleBlocks / kSelWarps];
+#pragma unroll
+  for (int u = 0; u < kSampleBlocks / kSelWarps; ++u) {   // all loads in flight together
+    const int blk = warp + u * kSelWarps;
+    v[u] = blk < nblk ? row[32 * ((blk * lpb) / nblk) + lane] : 0.0f;   // blk*lpb < 2^26
+  }
+  uint32_t lo_k = 0xFFFFFFFFu, hi_k = 0u;
+#pragma unroll
+  for (int u = 0; u < kSampleBlocks / kSelWarps; ++u) {
+    if (warp + u * kSelWarps < nblk) {
+      const uint32_t k = score_key(v[u]);
+      lo_k = min(lo_k, k);
+      hi_k = max(hi_k, k);
+    }
+  }
+  block_minmax(lo_k, hi_k, sm);
+  const float lo = key_to_float(lo_k), hi = key_to_float(hi_k);
+  if (!(hi > lo)) return lo;
+  const float scale = static_cast<float>(kBins) / (hi - lo);
+  if (!(scale < INFINITY)) return -INFINITY;
+  for (int i = tid; i < kBins; i += kSelThreads) sm.hist[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kSampleBlocks / kSelWarps; ++u)
+    if (warp + u * kSelWarps < nblk) atomicAdd(&sm.hist[lin_bin(v[u], lo, scale)], 1u);
+  __syncthreads();
+  const float rs = static_cast<float>(n_b) * static_cast<float>(S) / static_cast<float>(L);
+  uint32_t r = static_cast<uint32_t>(ceilf(rs + 6.0f * sqrtf(rs) + 8.0f));
+  if (r > static_cast<uint32_t>(S)) r = S;
+  {
+    const int b0 = 4 * (kSelThreads - 1 - tid);   // thread order runs over the bins top-down
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c += sm.hist[b0 + e];
+    uint32_t total;
+    uint32_t above = block_excl_scan(c, sm.scan, &total);
+    for (int e = 3; e >= 0; --e) {
+      const uint32_t h = sm.hist[b0 + e];
+      if (above < r && above + h >= r) sm.bcast[0] = b0 + e;
+      above += h;
+    }
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(sm.bcast[0]);
+  __syncthreads();
+  return bstar >= 1 ? lo + static_cast<float>(bstar - 1) / scale : -INFINITY;
+}
+
+// One compare pass over the row: (key, position) of every score >= t_lo goes
+// to the candidate buffer (warp-aggregated appends; entries past kCandCap are
+// counted, not stored).  With bulk copies the row arrives chunk by chunk in a
+// ring of shared-memory buffers.  Returns false if a wait timed out.
+__device__ bool gather_candidates(const float* row, int L, bool bulk, float t_lo, SelectSmem& sm,
+                                  int* status) {
   const int tid = threadIdx.x, lane = tid & 31;
+  const int n_chunks = (L + kChunk - 1) / kChunk;
+  volatile int never = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int s = c % kRing;
+    const int c0 = c * kChunk;
+    const int n_c = min(kChunk, L - c0);
+    const int n_bulk = bulk ? (n_c & ~3) : 0;        // floats that arrived by bulk copy
+    if (bulk) {
+      const bool ok = mbar_wait(smem_addr(&sm.full[s]), (c / kRing) & 1, &never);
+      if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+          atomicOr(status, 0x2 /* SAGA_STATUS_TIMEOUT */);
+          // let the copies still in flight land (bounded) before the CTA exits
+          for (int cc = c; cc < c + kRing && cc < n_chunks; ++cc)
+            mbar_wait(smem_addr(&sm.full[cc % kRing]), (cc / kRing) & 1, &never);
+        }
+        __syncthreads();
+        return false;
+      }
+    }
+    const int o = tid * kItems;
+    float v[8];
+    if (o + 7 < n_bulk) {
+      const float4 f0 = *reinterpret_cast<const float4*>(&sm.a.ring[s][o]);
+      const float4 f1 = *reinterpret_cast<const float4*>(&sm.a.ring[s][o + 4]);
+      v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+      v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int oe = o + e;
+        v[e] = oe < n_bulk ? sm.a.ring[s][oe] : (oe < n_c ? row[c0 + oe] : -INFINITY);
+      }
+    }
+    uint32_t fl = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (o + e < n_c && v[e] >= t_lo) fl |= 1u << e;
+    const uint32_t cnt = __popc(fl);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += y;
+    }
+    const uint32_t wsum = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t base = 0;
+    if (lane == 31 && wsum) base = atomicAdd(&sm.cand_n, wsum);
+    base = __shfl_sync(0xffffffffu, base, 31);
+    uint32_t w = base + incl - cnt;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if ((fl >> e) & 1u) {
+        if (w < static_cast<uint32_t>(kCandCap)) { sm.b.c.key[w] = score_key(v[e]); sm.b.c.pos[w] = c0 + o + e; }
+        ++w;
+      }
+    }
+    __syncthreads();                                   // ring buffer s is free again
+    if (bulk && tid == 0 && c + kRing < n_chunks) {
+      const int cn = c + kRing;
+      const int nb = min(kChunk, L - cn * kChunk) & ~3;
+      const uint32_t bar = smem_addr(&sm.full[s]);
+      if (nb > 0) {
+        mbar_arrive_expect_tx(bar, nb * 4);
+        bulk_load(smem_addr(sm.a.ring[s]), row + cn * kChunk, nb * 4, bar);
+      } else {
+        mbar_arrive(bar);
+      }
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+// Exact selection from the candidate buffer, which holds every score of the
+// row that can be among the top n_b (C entries, in no order): the n_b-th
+// largest key T; keys > T and the lowest-position ties are marked in a bitmap
+// of the row, and each kept candidate writes itself at slot = number of kept
+// positions before it.  Returns false (nothing written) if there were more
+// ties at T than the tie scratch holds.
+__device__ bool emit_from_candidates(int L, int n_b, int32_t* idx_out, float* logit_out,
+                                     SelectSmem& sm) {
+  const int tid = threadIdx.x;
+  const int C = static_cast<int>(sm.cand_n);
+  uint32_t need;
+  const uint32_t T = kth_largest(
+      [&](auto f) {
+        for (int i = tid; i < C; i += kSelThreads) f(sm.b.c.key[i]);
+      },
+      static_cast<uint32_t>(n_b), sm, &need);
+  const int W = (L + 31) / 32;
+  for (int i = tid; i < W; i += kSelThreads) sm.a.bm.bits[i] = 0;
+  if (tid == 0) sm.tie_n = 0;
+  __syncthreads();
+  for (int i = tid; i < C; i += kSelThreads) {
+    const uint32_t key = sm.b.c.key[i];
+    const int pos = sm.b.c.pos[i];
+    if (key > T) {
+      atomicOr(&sm.a.bm.bits[pos >> 5], 1u << (pos & 31));
+    } else if (key == T) {
+      const uint32_t t = atomicAdd(&sm.tie_n, 1u);
+      if (t < static_cast<uint32_t>(kBinKeys)) sm.bin_keys[t] = static_cast<uint32_t>(pos);
+    }
+  }
+  __syncthreads();
+  const uint32_t n_tie = sm.tie_n;
+  if (n_tie > static_cast<uint32_t>(kBinKeys)) return false;
+  for (uint32_t t = tid; t < n_tie; t += kSelThreads) {
+    const uint32_t pos = sm.bin_keys[t];
+    bool keep = true;
+    if (n_tie != need) {            // keep the `need` lowest positions among the ties
+      uint32_t rank = 0;
+      for (uint32_t u = 0; u < n_tie; ++u) rank += sm.bin_keys[u] < pos;
+      keep = rank < need;
+    }
+    if (keep) atomicOr(&sm.a.bm.bits[pos >> 5], 1u << (pos & 31));
+  }
+  __syncthreads();
+  // exclusive popcount prefix of the bitmap words (thread t owns a run of words)
+  const int wpt = (W + kSelThreads - 1) / kSelThreads;
+  const int w0 = tid * wpt, w1 = min(W, w0 + wpt);
+  uint32_t cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(sm.a.bm.bits[w]);
+  uint32_t total;
+  uint32_t run = block_excl_scan(cnt, sm.scan, &total);
+  for (int w = w0; w < w1; ++w) {
+    sm.a.bm.wpre[w] = run;
+    run += __popc(sm.a.bm.bits[w]);
+  }
+  __syncthreads();
+  for (int i = tid; i < C; i += kSelThreads) {
+    const int pos = sm.b.c.pos[i];
+    const uint32_t word = sm.a.bm.bits[pos >> 5];
+    const uint32_t bit = 1u << (pos & 31);
+    if (word & bit) {
+      const uint32_t slot = sm.a.bm.wpre[pos >> 5] + __popc(word & (bit - 1u));
+      idx_out[slot] = pos;
+      logit_out[slot] = key_to_float(sm.b.c.key[i]);
+    }
+  }
+  return true;
+}
+
+// Robust threshold: exact (T, ties needed) for the n_b-th largest score of the
+// row via an equal-width histogram of the whole row between its min and max.
+__device__ uint32_t robust_threshold(const float* row, int L, bool vec4, int n_b, uint32_t st_lo,
+                                     uint32_t st_hi, bool have_stats, int* status, SelectSmem& sm,
+                                     uint32_t* need_ties) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (!have_stats || st_lo > st_hi) {
+    uint32_t lo_k = 0xFFFFFFFFu, hi_k = 0u;
+    for (int i = tid; i < L; i += kSelThreads) {
+      const uint32_t key = score_key(row[i]);
+      lo_k = min(lo_k, key);
+      hi_k = max(hi_k, key);
+    }
+    block_minmax(lo_k, hi_k, sm);
+    st_lo = lo_k;
+    st_hi = hi_k;
+  }
+  const float lo = key_to_float(st_lo), hi = key_to_float(st_hi);
+  float scale = (hi > lo) ? static_cast<float>(kBins) / (hi - lo) : 0.0f;
+  if (!(scale < INFINITY)) scale = 0.0f;       // inf or NaN range: everything in bin 0
+
+  // pass A: histogram over equal-width bins
+  for (int i = tid; i < kBins; i += kSelThreads) sm.hist[i] = 0;
+  if (tid == 0) sm.cand_n = 0;
+  __syncthreads();
+  const int n_chunks4 = (L + 4 * kSelThreads - 1) / (4 * kSelThreads);
+  for (int c = 0; c < n_chunks4; ++c) {
+    const int base = c * 4 * kSelThreads + tid * 4;
+    if (vec4 && base + 3 < L) {
+      const float4 v = *reinterpret_cast<const float4*>(row + base);
+      atomicAdd(&sm.hist[lin_bin(v.x, lo, scale)], 1u);
+      atomicAdd(&sm.hist[lin_bin(v.y, lo, scale)], 1u);
+      atomicAdd(&sm.hist[lin_bin(v.z, lo, scale)], 1u);
+      atomicAdd(&sm.hist[lin_bin(v.w, lo, scale)], 1u);
+    } else {
+      for (int e = 0; e < 4; ++e)
+        if (base + e < L) atomicAdd(&sm.hist[lin_bin(row[base + e], lo, scale)], 1u);
+    }
+  }
+  __syncthreads();
+
+  // boundary bin: thread t owns bins [4*(511-t), +4), so thread order runs top-down
+  {
+    const int b0 = 4 * (kSelThreads - 1 - tid);
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c += sm.hist[b0 + e];
+    uint32_t total;
+    uint32_t above = block_excl_scan(c, sm.scan, &total);
+    for (int e = 3; e >= 0; --e) {
+      const uint32_t h = sm.hist[b0 + e];
+      if (above < static_cast<uint32_t>(n_b) && above + h >= static_cast<uint32_t>(n_b)) {
+        sm.bcast[0] = b0 + e; sm.bcast[1] = above; sm.bcast[2] = h;
+      }
+      above += h;
+    }
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(sm.bcast[0]);
+  const uint32_t above = sm.bcast[1];
+  const uint32_t in_bin = sm.bcast[2];
+  __syncthreads();
+
+  if (in_bin <= static_cast<uint32_t>(kCandCap)) {
+    // pass B: keys of the boundary bin
+    for (int c = 0; c < n_chunks4; ++c) {
+      const int base = c * 4 * kSelThreads + tid * 4;
+      float v[4];
+      if (vec4 && base + 3 < L) {
+        const float4 f = *reinterpret_cast<const float4*>(row + base);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+      } else {
+        for (int e = 0; e < 4; ++e) v[e] = (base + e < L) ? row[base + e] : 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool pred = (base + e < L) && lin_bin(v[e], lo, scale) == bstar;
+        const uint32_t m = __ballot_sync(0xffffffffu, pred);
+        if (m) {
+          const int leader = __ffs(m) - 1;
+          uint32_t slot = 0;
+          if (lane == leader) slot = atomicAdd(&sm.cand_n, static_cast<uint32_t>(__popc(m)));
+          slot = __shfl_sync(0xffffffffu, slot, leader);
+          if (pred) sm.b.c.key[slot + __popc(m & ((1u << lane) - 1u))] = score_key(v[e]);
+        }
+      }
+    }
+    __syncthreads();
+    const int n_cand = static_cast<int>(sm.cand_n);
+    return radix_select(
+        [&](auto f) {
+          for (int i = tid; i < n_cand; i += kSelThreads) f(sm.b.c.key[i]);
+        },
+        static_cast<uint32_t>(n_b) - above, sm, need_ties);
+  }
+  // flat row: exact radix select over the whole row
+  if (tid == 0) atomicOr(status, 0x100 /* SAGA_STATUS_INFO_EXACT_FALLBACK */);
+  return radix_select(
+      [&](auto f) {
+        for (int i = tid; i < L; i += kSelThreads) f(score_key(row[i]));
+      },
+      static_cast<uint32_t>(n_b), sm, need_ties);
+}
+
+// Ordered compare pass: keep key > T and the first `need` ties, positions ascending.
+__device__ void emit_by_threshold(const float* row, int L, bool vec4, uint32_t T, uint32_t need,
+                                  int32_t* idx_out, float* logit_out, SelectSmem& sm) {
+  const int tid = threadIdx.x;
+  uint32_t run_gt = 0, run_tie = 0;
+  const int n_chunks = (L + kChunk - 1) / kChunk;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int base = c * kChunk + tid * kItems;
+    float v[8];
+    load8(row, base, L, vec4, v);
+    uint32_t gt = 0, tie = 0;
+#pragma unroll
+    for (int e = 0; e < kItems; ++e) {
+      if (base + e < L) {
+        const uint32_t key = score_key(v[e]);
+        if (key > T) gt |= 1u << e;
+        else if (key == T) tie |= 1u << e;
+      }
+    }
+    uint32_t total;
+    const uint32_t excl = block_excl_scan((static_cast<uint32_t>(__popc(tie)) << 16) | __popc(gt),
+                                          sm.scan, &total);
+    uint32_t tr = run_tie + (excl >> 16);
+    uint32_t w = run_gt + (excl & 0xFFFFu) + min(need, tr);
+#pragma unroll
+    for (int e = 0; e < kItems; ++e) {
+      bool sel = (gt >> e) & 1u;
+      if ((tie >> e) & 1u) { sel = tr < need; ++tr; }
+      if (sel) {
+        idx_out[w] = base + e;
+        logit_out[w] = v[e];
+        ++w;
+      }
+    }
+    run_gt += total & 0xFFFFu;
+    run_tie += total >> 16;
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2)
+select_kernel(const SelectParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  const int tid = threadIdx.x;
   const int bj = blockIdx.x;
   const int b = bj / p.h_q;
   const int L = p.seq_lens[b];
@@ -296,171 +630,71 @@ select_combine_kernel(const SelectParams p) {
   int32_t* idx_out = p.sel_idx + static_cast<long long>(bj) * N;
   float* logit_out = p.sel_logit + static_cast<long long>(bj) * N;
   const float* row = p.z + static_cast<long long>(bj) * p.z_stride;
+  const bool vec4 = p.z_vec4 != 0;
+  const bool valid = L >= 1 && L <= p.L_max;
+  const int n_b = N < L ? N : L;
+  // the fast path: candidates through shared memory, bitmap emission
+  const bool fast = valid && n_b < L && L <= kMaxBitmapL && n_b <= kCandCap / 2;
+  const bool bulk = fast && vec4;
 
   uint32_t st_lo = 0xFFFFFFFFu, st_hi = 0u;
   if (p.stat_min != nullptr) { st_lo = p.stat_min[bj]; st_hi = p.stat_max[bj]; }
+  if (tid == 0) {
+    sm.cand_n = 0;
+    if (bulk) {                     // start streaming the row before anything else
+      for (int s = 0; s < kRing; ++s) mbar_init(smem_addr(&sm.full[s]), 1);
+      fence_mbar_init();
+      const int n_chunks = (L + kChunk - 1) / kChunk;
+      for (int c = 0; c < kRing && c < n_chunks; ++c) {
+        const int nb = min(kChunk, L - c * kChunk) & ~3;
+        const uint32_t bar = smem_addr(&sm.full[c]);
+        if (nb > 0) {
+          mbar_arrive_expect_tx(bar, nb * 4);
+          bulk_load(smem_addr(sm.a.ring[c]), row + c * kChunk, nb * 4, bar);
+        } else {
+          mbar_arrive(bar);
+        }
+      }
+    }
+  }
   __syncthreads();
-  if (tid == 0 && p.stat_min != nullptr) {    // leave the statistics ready for the next call
-    p.stat_min[bj] = 0xFFFFFFFFu;
-    p.stat_max[bj] = 0u;
+  if (tid == 0) {
+    if (p.stat_min != nullptr) {   // leave the statistics ready for the next call
+      p.stat_min[bj] = 0xFFFFFFFFu;
+      p.stat_max[bj] = 0u;
+    }
+    if (p.gather_count != nullptr) p.gather_count[bj] = 0u;
   }
 
-  if (L < 1 || L > p.L_max) {
+  if (!valid) {
     if (tid == 0) atomicOr(p.status, 0x1 /* SAGA_STATUS_BAD_SEQ_LEN */);
     for (int r = tid; r < N; r += kSelThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
-    if (p.out != nullptr)
-      for (int e = tid; e < D; e += kSelThreads) p.out[static_cast<long long>(bj) * D + e] = __float2bfloat16_rn(0.0f);
     return;
   }
-  const int n_b = N < L ? N : L;
-  const bool dense = (n_b == L);
 
-  auto load_z = [&](int i) -> float { return row[i]; };
-
-  uint32_t T = 0, need_ties = 0;
-  if (!dense) {
-    // ---- range of the row: from the score pass, else one min/max pass
-    if (p.stat_min == nullptr || st_lo > st_hi) {
-      uint32_t lo_k = 0xFFFFFFFFu, hi_k = 0u;
-      for (int i = tid; i < L; i += kSelThreads) {
-        const uint32_t key = score_key(load_z(i));
-        lo_k = min(lo_k, key);
-        hi_k = max(hi_k, key);
-      }
-      st_lo = block_min_u32(lo_k, sm.scan);
-      st_hi = block_max_u32(hi_k, sm.scan);
-    }
-    const float lo = key_to_float(st_lo), hi = key_to_float(st_hi);
-    float scale = (hi > lo) ? static_cast<float>(kBins) / (hi - lo) : 0.0f;
-    if (!(scale < INFINITY)) scale = 0.0f;       // inf or NaN range: everything in bin 0
-
-    // ---- pass A: histogram over equal-width bins
-    for (int i = tid; i < kBins; i += kSelThreads) sm.hist[i] = 0;
-    if (tid == 0) sm.cand_n = 0;
-    __syncthreads();
-    const int n_chunks4 = (L + 4 * kSelThreads - 1) / (4 * kSelThreads);
-    for (int c = 0; c < n_chunks4; ++c) {
-      const int base = c * 4 * kSelThreads + tid * 4;
-      if (p.z_vec4 && base + 3 < L) {
-        const float4 v = *reinterpret_cast<const float4*>(row + base);
-        atomicAdd(&sm.hist[lin_bin(v.x, lo, scale)], 1u);
-        atomicAdd(&sm.hist[lin_bin(v.y, lo, scale)], 1u);
-        atomicAdd(&sm.hist[lin_bin(v.z, lo, scale)], 1u);
-        atomicAdd(&sm.hist[lin_bin(v.w, lo, scale)], 1u);
-      } else {
-        for (int e = 0; e < 4; ++e)
-          if (base + e < L) atomicAdd(&sm.hist[lin_bin(load_z(base + e), lo, scale)], 1u);
-      }
-    }
-    __syncthreads();
-
-    // ---- boundary bin: thread t owns bins [4*(511-t), +4), so thread order runs top-down
-    {
-      const int b0 = 4 * (kSelThreads - 1 - tid);
-      uint32_t c = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) c += sm.hist[b0 + e];
-      uint32_t total;
-      uint32_t above = block_excl_scan(c, sm.scan, &total);
-      for (int e = 3; e >= 0; --e) {
-        const uint32_t h = sm.hist[b0 + e];
-        if (above < static_cast<uint32_t>(n_b) && above + h >= static_cast<uint32_t>(n_b)) {
-          sm.bcast[0] = b0 + e; sm.bcast[1] = above; sm.bcast[2] = h;
-        }
-        above += h;
-      }
-    }
-    __syncthreads();
-    const int bstar = static_cast<int>(sm.bcast[0]);
-    const uint32_t above = sm.bcast[1];
-    const uint32_t in_bin = sm.bcast[2];
-    __syncthreads();
-
-    if (in_bin <= static_cast<uint32_t>(kCandCap)) {
-      // ---- pass B: keys of the boundary bin
-      for (int c = 0; c < n_chunks4; ++c) {
-        const int base = c * 4 * kSelThreads + tid * 4;
-        float v[4];
-        if (p.z_vec4 && base + 3 < L) {
-          const float4 f = *reinterpret_cast<const float4*>(row + base);
-          v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-        } else {
-          for (int e = 0; e < 4; ++e) v[e] = (base + e < L) ? load_z(base + e) : 0.0f;
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool pred = (base + e < L) && lin_bin(v[e], lo, scale) == bstar;
-          const uint32_t m = __ballot_sync(0xffffffffu, pred);
-          if (m) {
-            const int leader = __ffs(m) - 1;
-            uint32_t slot = 0;
-            if (lane == leader) slot = atomicAdd(&sm.cand_n, static_cast<uint32_t>(__popc(m)));
-            slot = __shfl_sync(0xffffffffu, slot, leader);
-            if (pred) sm.u.cand[slot + __popc(m & ((1u << lane) - 1u))] = score_key(v[e]);
-          }
-        }
-      }
+  if (n_b == L) {
+    // every position is selected (dense softmax attention)
+    for (int i = tid; i < L; i += kSelThreads) { idx_out[i] = i; logit_out[i] = row[i]; }
+  } else {
+    bool done = false;
+    if (fast) {
+      const float t_lo = (L <= kChunk) ? -INFINITY : sample_bound(row, L, n_b, sm);
+      const bool ok = gather_candidates(row, L, bulk, t_lo, sm, p.status);
+      if (!ok) return;                                   // timed out: status already set
+      const uint32_t C = sm.cand_n;
+      if (C >= static_cast<uint32_t>(n_b) && C <= static_cast<uint32_t>(kCandCap))
+        done = emit_from_candidates(L, n_b, idx_out, logit_out, sm);
       __syncthreads();
-      const int n_cand = static_cast<int>(sm.cand_n);
-      T = radix_select([&](int i) { return sm.u.cand[i]; }, n_cand,
-                       static_cast<uint32_t>(n_b) - above, sm, &need_ties);
-    } else {
-      // ---- flat row: exact radix select over the whole row
-      if (tid == 0) atomicOr(p.status, 0x100 /* SAGA_STATUS_INFO_EXACT_FALLBACK */);
-      T = radix_select([&](int i) { return score_key(load_z(i)); }, L,
-                       static_cast<uint32_t>(n_b), sm, &need_ties);
     }
-  }
-
-  // ---- pass C: compare and compact in position order
-  uint32_t run_gt = 0, run_tie = 0;
-  float m_local = -INFINITY;
-  const int n_chunks = (L + kChunk - 1) / kChunk;
-  for (int c = 0; c < n_chunks; ++c) {
-    const int base = c * kChunk + tid * kItems;
-    float v[kItems];
-    if (p.z_vec4 && base + kItems - 1 < L) {
-      const float4 f0 = *reinterpret_cast<const float4*>(row + base);
-      const float4 f1 = *reinterpret_cast<const float4*>(row + base + 4);
-      v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
-      v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < kItems; ++e) v[e] = (base + e < L) ? load_z(base + e) : 0.0f;
+    if (!done) {
+      if (tid == 0) atomicOr(p.status, 0x200 /* SAGA_STATUS_INFO_ROBUST_PATH */);
+      uint32_t need;
+      const uint32_t T = robust_threshold(row, L, vec4, n_b, st_lo, st_hi, p.stat_min != nullptr,
+                                          p.status, sm, &need);
+      emit_by_threshold(row, L, vec4, T, need, idx_out, logit_out, sm);
     }
-    uint32_t gt_mask = 0, tie_mask = 0;
-#pragma unroll
-    for (int e = 0; e < kItems; ++e) {
-      if (base + e < L) {
-        const uint32_t key = score_key(v[e]);
-        if (dense || key > T) gt_mask |= 1u << e;
-        else if (key == T) tie_mask |= 1u << e;
-      }
-    }
-    const uint32_t packed = (static_cast<uint32_t>(__popc(tie_mask)) << 16) | __popc(gt_mask);
-    uint32_t total;
-    const uint32_t excl = block_excl_scan(packed, sm.scan, &total);
-    uint32_t tr = run_tie + (excl >> 16);
-    uint32_t w = run_gt + (excl & 0xFFFFu) + min(need_ties, tr);
-#pragma unroll
-    for (int e = 0; e < kItems; ++e) {
-      bool sel = (gt_mask >> e) & 1u;
-      if ((tie_mask >> e) & 1u) { sel = tr < need_ties; ++tr; }
-      if (sel) {
-        idx_out[w] = base + e;
-        logit_out[w] = v[e];
-        m_local = fmaxf(m_local, v[e]);
-        ++w;
-      }
-    }
-    run_gt += total & 0xFFFFu;
-    run_tie += total >> 16;
   }
   for (int r = n_b + tid; r < N; r += kSelThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
-  if (p.out == nullptr) return;
-  const float m = block_max(m_local, sm.fred);   // also orders the list writes above
-
-  combine_rows<D>(p, bj, idx_out, logit_out, n_b, L, m, sm);
 }
 
 }  // namespace saga

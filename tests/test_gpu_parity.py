@@ -155,8 +155,10 @@ def test_duplicate_keys_ties_go_to_lowest_index():
 
 
 def test_all_equal_scores_take_lowest_positions():
-    B, L, h_q, h_k, h_v, d, N = 2, 5000, 4, 1, 1, 128, 777
-    inp = make_raw(8, B, L, [L, 4000], h_q, h_k, h_v, d)
+    # row 0 is too long for the candidate buffer and too flat for the histogram:
+    # it takes the whole-row radix select; row 1 fits the buffer directly
+    B, L, h_q, h_k, h_v, d, N = 2, 20000, 4, 1, 1, 128, 777
+    inp = make_raw(8, B, L, [L, 5000], h_q, h_k, h_v, d)
     inp.k_cache[:] = inp.k_cache[:, :, :1]            # one key everywhere: every score equal
     dec = SagaDecoder(B, L, h_q, h_k, h_v, d, N)
     out, idx, logit, st = run_decode(dec, *_dev(inp), N)
@@ -289,7 +291,7 @@ def test_deterministic_and_host_entry_point():
     n0 = dec.launch_count()
     dec.attn_host(q_h, k, v, l_h, spec.N, o_h)
     assert dec.status() == 0
-    assert dec.launch_count() - n0 == 2
+    assert dec.launch_count() - n0 == 3   # score, select, gather
     assert torch.equal(o_h, a.cpu())
 
 
