@@ -71,6 +71,7 @@ extern "C" {
 #define SAGA_ERR_UNSUPPORTED  2  /* valid but not built: d not in {64,128}, g > 64, wrong GPU */
 #define SAGA_ERR_CUDA         3  /* a CUDA runtime/driver call failed */
 #define SAGA_ERR_DEVICE       4  /* saga_decode_status found an error bit set */
+#define SAGA_ERR_SCRATCH_TOO_SMALL 5  /* saga_combine_noalloc: sizes exceed its fixed scratch */
 
 /* Device status bits (saga_decode_status). */
 #define SAGA_STATUS_BAD_SEQ_LEN   0x1   /* some seq_lens[b] outside [1, L_max]: row zeroed */
@@ -150,6 +151,28 @@ SAGA_API int saga_select(saga_handle h, const float* scores, int scores_stride,
 SAGA_API int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
                  const void* v_cache, const int32_t* seq_lens, int h_q, int h_v,
                  int head_dim, int N, void* out);
+
+/* saga_combine_noalloc -- stages S3+S4 (as saga_combine) without a handle and without
+ * allocating anything.  The paper has no counterpart: it exists for callers that cannot
+ * allocate device memory (a serving engine whose memory manager owns the whole device, a
+ * process under a hard memory cap, code running inside graph capture or an allocator
+ * callback), which therefore cannot create a handle.  Inputs and outputs are the caller's
+ * device arrays, with the layouts above: sel_idx / sel_logit [batch][h_q][N], v_cache
+ * [batch][h_v][max_seq_len][head_dim], seq_lens [batch], out bf16 [batch][h_q][head_dim];
+ * cuda_stream is a cudaStream_t (NULL = legacy default stream).  The kernel's scratch (a
+ * status word, per-row merge counters and per-chunk softmax partials) is a fixed 4 MiB array
+ * inside the library, reserved on every GPU that loads the library until the process exits.
+ * Limit: 256 + round_up(4*batch*h_q, 256) + round_up(4*batch*h_q*ceil(min(N,max_seq_len)/256)
+ * *(head_dim+2), 256) <= 4 MiB (e.g. batch*h_q = 192 rows with N = 1024 and head_dim = 128
+ * uses 0.4 MiB), else SAGA_ERR_SCRATCH_TOO_SMALL and nothing runs.  The first call on each
+ * device looks up the array's device address; make that first call before any stream
+ * capture.  Every call clears the part of the array that must start at zero and reuses the
+ * rest, so calls that can overlap on the GPU (different streams) race and must not be issued
+ * concurrently.  Rows with seq_lens[b] outside [1, max_seq_len] get zeros.  Asynchronous. */
+SAGA_API int saga_combine_noalloc(const int32_t* sel_idx, const float* sel_logit,
+                                  const void* v_cache, const int32_t* seq_lens, int batch,
+                                  int max_seq_len, int h_q, int h_v, int head_dim, int N,
+                                  void* out, void* cuda_stream);
 
 /* Synchronise the handle's stream, then return (in *device_status) and clear
  * the device status word.  Returns SAGA_ERR_DEVICE if an error bit

@@ -17,7 +17,7 @@ import torch
 from . import _lib
 from ._lib import SagaError, load  # noqa: F401
 
-__all__ = ["SagaDecoder", "SagaError", "load"]
+__all__ = ["SagaDecoder", "SagaError", "load", "combine_noalloc"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -202,3 +202,33 @@ class SagaDecoder:
             self.close()
         except Exception:
             pass
+
+
+def combine_noalloc(sel_idx, sel_logit, v_cache, seq_lens, out):
+    """Softmax over a selection and the gathered P.V (stages S3 + S4) without a handle.
+
+    For callers that cannot allocate device memory -- e.g. a serving engine whose memory
+    manager owns the whole device, or a process under a hard memory cap -- and so cannot
+    create a SagaDecoder (its workspace is allocated).  This function allocates nothing, not
+    even the output: ``out`` (bf16 [B, h_q, d]) must be supplied.  The library keeps the
+    kernel's scratch in a fixed 4 MiB array of its own; problems that do not fit raise
+    SagaError (SAGA_ERR_SCRATCH_TOO_SMALL).  The first call on a device should come before
+    any stream capture, and calls on different streams must not overlap on the GPU.
+    sel_idx / sel_logit: [B, h_q, N] (index -1 = padding); v_cache: [B, h_v, L_max, d] bf16;
+    seq_lens: [B] int32.  Runs on the current stream, asynchronously.
+    """
+    lib = load()
+    B, h_q, N = sel_idx.shape
+    _need(sel_idx, "sel_idx", torch.int32, (B, h_q, N), "cuda")
+    _need(sel_logit, "sel_logit", torch.float32, (B, h_q, N), "cuda")
+    _need(v_cache, "v_cache", torch.bfloat16, device="cuda")
+    if v_cache.dim() != 4 or v_cache.shape[0] != B:
+        raise ValueError("v_cache must be [B, h_v, L_max, d]")
+    _, h_v, L_max, d = v_cache.shape
+    _need(seq_lens, "seq_lens", torch.int32, (B,), "cuda")
+    _need(out, "out", torch.bfloat16, (B, h_q, d), "cuda")
+    stream = torch.cuda.current_stream(out.device).cuda_stream
+    _lib.check("saga_combine_noalloc", lib.saga_combine_noalloc(
+        _ptr(sel_idx), _ptr(sel_logit), _ptr(v_cache), _ptr(seq_lens), B, L_max, h_q, h_v, d, N,
+        _ptr(out), ctypes.c_void_p(stream)))
+    return out

@@ -10,6 +10,7 @@ SAGA_ERR_INVALID_ARG = 1
 SAGA_ERR_UNSUPPORTED = 2
 SAGA_ERR_CUDA = 3
 SAGA_ERR_DEVICE = 4
+SAGA_ERR_SCRATCH_TOO_SMALL = 5
 SAGA_STATUS_BAD_SEQ_LEN = 0x1
 SAGA_STATUS_TIMEOUT = 0x2
 SAGA_STATUS_BAD_INDEX = 0x4
@@ -30,6 +31,7 @@ SIGNATURES = {
     "saga_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I]),
     "saga_select": (_I, [_P, _P, _I, _P, _I, _I, _P, _P]),
     "saga_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "saga_combine_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "saga_decode_status": (_I, [_P, ctypes.POINTER(_I)]),
     "saga_decode_launch_count": (_I, [_P, ctypes.POINTER(ctypes.c_longlong)]),
     "saga_decode_profile": (_I, [_P, _I, _I]),

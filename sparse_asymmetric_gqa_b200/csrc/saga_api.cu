@@ -272,6 +272,8 @@ const char* saga_decode_error_string(int code) {
     case SAGA_ERR_UNSUPPORTED: return "unsupported configuration or device";
     case SAGA_ERR_CUDA: return "CUDA call failed";
     case SAGA_ERR_DEVICE: return "device reported an error (see saga_decode_status)";
+    case SAGA_ERR_SCRATCH_TOO_SMALL:
+      return "problem too large for the fixed scratch of saga_combine_noalloc (4 MiB)";
     default: return "unknown error code";
   }
 }
@@ -503,6 +505,101 @@ int saga_decode_free(saga_handle h) {
   }
   delete h;
   return rc;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// saga_combine_noalloc -- softmax over a selection and the gathered P.V (stages S3 + S4) for
+// callers that cannot allocate device memory.
+//
+// Who needs it: code that must not call cudaMalloc -- for example a serving engine whose memory
+// manager reserves all device memory up front and hands out only its own pool, a process sharing
+// the GPU under a hard memory cap, or a caller inside CUDA-graph capture or an allocator callback
+// where an allocation would fail or deadlock.  Such callers cannot create a saga_decode handle,
+// because the handle allocates its workspace.  This entry point needs no handle: the only scratch
+// the gather kernel uses (per-chunk softmax partials, per-row merge counters and a status word)
+// lives in the fixed array below, which is part of the library image and is reserved on every GPU
+// that loads the library until the process exits.
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// The device address of g_noalloc_scratch on device `dev` (the current device).  Host code may
+// not pass the symbol itself to a kernel: on the host it names a host-side stand-in.
+int noalloc_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SAGA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return SAGA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+  return SAGA_OK;
+}
+
+size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+int saga_combine_noalloc(const int32_t* sel_idx, const float* sel_logit, const void* v_cache,
+                         const int32_t* seq_lens, int batch, int max_seq_len, int h_q, int h_v,
+                         int head_dim, int N, void* out, void* cuda_stream) {
+  if (!sel_idx || !sel_logit || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (batch < 1 || max_seq_len < 1 || h_q < 1 || h_v < 1 || N < 1) return SAGA_ERR_INVALID_ARG;
+  if (h_q % h_v != 0) return SAGA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return SAGA_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(batch) * h_q;
+  if (rows > (1ll << 30)) return SAGA_ERR_INVALID_ARG;
+  const int slots = N < max_seq_len ? N : max_seq_len;
+  const int chunks = (slots + kGatherRows - 1) / kGatherRows;
+  if (chunks > 65535) return SAGA_ERR_SCRATCH_TOO_SMALL;
+  // scratch layout: status word | merge counters [rows] | partials [rows][chunks][head_dim + 2]
+  const size_t status_bytes = 256;
+  const size_t counter_bytes = al256(static_cast<size_t>(rows) * sizeof(uint32_t));
+  const size_t part_bytes = al256(static_cast<size_t>(rows) * chunks * (head_dim + 2) * sizeof(float));
+  if (status_bytes + counter_bytes + part_bytes > kNoAllocScratchBytes) return SAGA_ERR_SCRATCH_TOO_SMALL;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGA_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  if (int rc = noalloc_scratch(dev, &scratch)) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  // the status word and the counters must start at zero; the array keeps the last call's contents
+  if (cudaMemsetAsync(scratch, 0, status_bytes + counter_bytes, stream) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+
+  GatherParams p;
+  p.sel_idx = sel_idx;
+  p.sel_logit = sel_logit;
+  p.seq_lens = seq_lens;
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.h_q = h_q;
+  p.h_v = h_v;
+  p.g_v = h_q / h_v;
+  p.L_max = max_seq_len;
+  p.N = N;
+  p.status = reinterpret_cast<int*>(scratch);
+  p.counter = reinterpret_cast<uint32_t*>(scratch + status_bytes);
+  p.partial = reinterpret_cast<float*>(scratch + status_bytes + counter_bytes);
+  p.max_chunks = chunks;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(chunks));
+  if (head_dim == 64)
+    gather_kernel<64><<<grid, kGatherThreads, 0, stream>>>(p);
+  else
+    gather_kernel<128><<<grid, kGatherThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 }  // extern "C"
