@@ -76,11 +76,14 @@ extern "C" {
 /* Device status bits (saga_decode_status). */
 #define SAGA_STATUS_BAD_SEQ_LEN   0x1   /* some seq_lens[b] outside [1, L_max]: row zeroed */
 #define SAGA_STATUS_TIMEOUT       0x2   /* an internal pipeline wait ran out: results invalid */
-#define SAGA_STATUS_BAD_INDEX     0x4   /* saga_combine got an index >= L_b: that slot ignored */
+#define SAGA_STATUS_BAD_INDEX     0x4   /* saga_combine got an index >= L_b (that slot ignored), or
+                                           a candidate position was outside [0, L_b) */
 #define SAGA_STATUS_INFO_EXACT_FALLBACK 0x100  /* informational: a row needed the full radix
                                                    select (very flat score rows); not an error */
 #define SAGA_STATUS_INFO_ROBUST_PATH 0x200     /* informational: a row's sampled threshold bound
-                                                   missed and the histogram path ran; not an error */
+                                                   missed (or the row was too long or too flat for
+                                                   the candidate list) and the exact whole-row
+                                                   path ran; not an error */
 
 typedef struct saga_ctx* saga_handle;
 
@@ -184,11 +187,13 @@ SAGA_API int saga_decode_status(saga_handle h, int* device_status);
 SAGA_API int saga_decode_launch_count(saga_handle h, long long* count);
 
 /* Profiling: when enabled, each decode call records CUDA events around its
- * score kernel and around the whole call on the handle's stream (up to
- * max_calls calls; inside CUDA-graph capture the records become graph nodes,
- * so every replay re-records them).  saga_decode_profile_read synchronises and
- * returns the summed milliseconds and the number of calls recorded, then
- * starts counting calls from zero again. */
+ * score pass (threshold + score kernels) and around the whole call on the
+ * handle's stream (up to max_calls calls; inside CUDA-graph capture the
+ * records become graph nodes, so every replay re-records them; the events
+ * live until the handle is freed).  Disabling stops recording and keeps the
+ * events.  saga_decode_profile_read synchronises and returns the summed
+ * milliseconds and the number of calls recorded, then starts counting calls
+ * from zero again. */
 SAGA_API int saga_decode_profile(saga_handle h, int enable, int max_calls);
 SAGA_API int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms,
                              int* n_calls);

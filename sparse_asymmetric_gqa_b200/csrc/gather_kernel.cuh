@@ -49,6 +49,7 @@ template <int D>
 __global__ void __launch_bounds__(kGatherThreads)
 gather_kernel(const GatherParams p) {
   __shared__ GatherSmem<D> sm;
+  pdl_wait();                        // the selection lists are complete (no-op without PDL)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bj = blockIdx.x;
   const int chunk = blockIdx.y;

@@ -192,6 +192,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Let the next kernel in the stream (launched with programmatic stream
+// serialization) start now; it must still wait before reading our results.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the preceding kernel in the stream has completed and its memory
+// operations are visible (a no-op when launched without the attribute).
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- misc
 // Order-preserving map fp32 -> uint32 (larger float -> larger key).  Callers
 // canonicalise -0 to +0 first.

@@ -16,6 +16,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "saga.h"
@@ -23,6 +24,8 @@
 #include "score_kernel.cuh"
 #include "select_kernel.cuh"
 #include "gather_kernel.cuh"
+#include "threshold_kernel.cuh"
+#include "topn_kernel.cuh"
 
 using namespace saga;
 
@@ -83,6 +86,11 @@ struct saga_ctx {
   __nv_bfloat16* q_stage = nullptr;
   __nv_bfloat16* out_stage = nullptr;
   int32_t* lens_stage = nullptr;
+  float scale = 0.0f;             // 1/sqrt(d) rounded to fp32
+  float* t_lo = nullptr;          // candidate thresholds [rows]
+  uint32_t* cand_count = nullptr; // candidates appended per row [rows]
+  uint32_t* cand_key = nullptr;   // candidate lists [rows][kTopnCap] (null: lists not kept)
+  int32_t* cand_pos = nullptr;
   float* partial = nullptr;       // gather partials [rows][max_chunks][d + 2]
   uint32_t* counter = nullptr;    // gather merge counters [rows]
   int max_chunks = 0;
@@ -100,28 +108,54 @@ int set_smem_attrs_once() {
   static std::once_flag once;
   std::call_once(once, []() {
     cudaError_t e = cudaSuccess;
-#define SAGA_ATTR(D, NP)                                                                       \
-  if (e == cudaSuccess)                                                                        \
-    e = cudaFuncSetAttribute(score_kernel<D, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             ScoreShape<D, NP>::kSmemBytes);
+#define SAGA_ATTR(D, NP)                                                                          \
+  if (e == cudaSuccess)                                                                           \
+    e = cudaFuncSetAttribute(score_kernel<D, NP, false>,                                          \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes); \
+  if (e == cudaSuccess)                                                                           \
+    e = cudaFuncSetAttribute(score_kernel<D, NP, true>,                                           \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes);
     SAGA_ATTR(64, 16) SAGA_ATTR(64, 32) SAGA_ATTR(64, 48) SAGA_ATTR(64, 64)
     SAGA_ATTR(128, 16) SAGA_ATTR(128, 32) SAGA_ATTR(128, 48) SAGA_ATTR(128, 64)
 #undef SAGA_ATTR
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sizeof(SelectSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kTopnSmemBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kTopnSmemBytes));
     rc = (e == cudaSuccess) ? 0 : 1;
   });
   return rc;
 }
 
-template <int D, int NP>
-cudaError_t launch_score_t(saga_ctx* h, const CUtensorMap& mk, const CUtensorMap& mq,
-                           const ScoreParams& p, int grid) {
-  score_kernel<D, NP><<<grid, kScoreThreads, ScoreShape<D, NP>::kSmemBytes, h->stream>>>(mk, mq, p);
-  return cudaGetLastError();
+// Launch on the handle's stream; with `pdl` the kernel may start before the
+// previous kernel in the stream has finished (it waits in-kernel before it
+// reads that kernel's results: programmatic dependent launch).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(saga_ctx* h, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = h->stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) ++h->launches;
+  return e;
 }
 
+// Score pass.  z == nullptr: candidate mode (thresholds from h->t_lo, lists in
+// the workspace, launched as a dependent of the threshold kernel); otherwise
+// every score goes to z.
 int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
                  float* z, long long z_stride, bool stats) {
   CUtensorMap mk, mq;
@@ -129,11 +163,18 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
   const uint64_t q_rows = static_cast<uint64_t>(h->batch) * h->h_q;
   if (!encode_bf16_2d(&mk, k_cache, k_rows, h->d, kTileM)) return SAGA_ERR_CUDA;
   if (!encode_bf16_2d(&mq, q, q_rows, h->d, h->npad)) return SAGA_ERR_CUDA;
+  const bool cand = (z == nullptr);
   ScoreParams p;
+  std::memset(&p, 0, sizeof(p));
   p.seq_lens = seq_lens;
   p.z = z;
-  p.stat_min = stats ? h->stat_min : nullptr;
-  p.stat_max = stats ? h->stat_max : nullptr;
+  p.t_lo = h->t_lo;
+  p.cand_count = h->cand_count;
+  p.cand_key = h->cand_key;
+  p.cand_pos = h->cand_pos;
+  p.cand_cap = kTopnCap;
+  p.stat_min = (stats && !cand) ? h->stat_min : nullptr;
+  p.stat_max = (stats && !cand) ? h->stat_max : nullptr;
   p.status = h->status;
   p.B = h->batch;
   p.h_q = h->h_q;
@@ -141,19 +182,71 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
   p.g = h->g;
   p.L_max = h->max_seq_len;
   p.z_stride = z_stride;
-  p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d)));
+  p.scale = h->scale;
   const long long max_units =
       static_cast<long long>(h->batch) * h->h_k * ((h->max_seq_len + kTileM - 1) / kTileM);
   const int grid = static_cast<int>(max_units < h->num_sms ? max_units : h->num_sms);
   cudaError_t e = cudaErrorInvalidValue;
-#define SAGA_CASE(D, NP) \
-  if (h->d == D && h->npad == NP) e = launch_score_t<D, NP>(h, mk, mq, p, grid);
+#define SAGA_CASE(D, NP)                                                                       \
+  if (h->d == D && h->npad == NP)                                                              \
+    e = cand ? launch(h, score_kernel<D, NP, true>, dim3(grid), dim3(kScoreThreads),           \
+                      ScoreShape<D, NP>::kSmemBytes, true, mk, mq, p)                          \
+             : launch(h, score_kernel<D, NP, false>, dim3(grid), dim3(kScoreThreads),          \
+                      ScoreShape<D, NP>::kSmemBytes, false, mk, mq, p);
   SAGA_CASE(64, 16) SAGA_CASE(64, 32) SAGA_CASE(64, 48) SAGA_CASE(64, 64)
   SAGA_CASE(128, 16) SAGA_CASE(128, 32) SAGA_CASE(128, 48) SAGA_CASE(128, 64)
 #undef SAGA_CASE
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
-  ++h->launches;
-  return SAGA_OK;
+  return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
+}
+
+int launch_threshold(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
+                     int N) {
+  ThresholdParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.seq_lens = seq_lens;
+  p.h_q = h->h_q;
+  p.h_k = h->h_k;
+  p.g = h->g;
+  p.L_max = h->max_seq_len;
+  p.N = N;
+  p.cand_cap = kTopnCap;
+  p.scale = h->scale;
+  p.t_lo = h->t_lo;
+  const dim3 grid(h->batch * h->h_q);
+  const cudaError_t e = (h->d == 64)
+      ? launch(h, threshold_kernel<64>, grid, dim3(kThrThreads), 0, false, p)
+      : launch(h, threshold_kernel<128>, grid, dim3(kThrThreads), 0, false, p);
+  return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
+}
+
+int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens, int N,
+                int32_t* sel_idx, float* sel_logit) {
+  TopnParams p;
+  p.cand_key = h->cand_key;
+  p.cand_pos = h->cand_pos;
+  p.cand_count = h->cand_count;
+  p.cand_cap = kTopnCap;
+  p.gather_count = h->counter;
+  p.seq_lens = seq_lens;
+  p.h_q = h->h_q;
+  p.h_k = h->h_k;
+  p.g = h->g;
+  p.L_max = h->max_seq_len;
+  p.N = N;
+  p.sel_idx = sel_idx;
+  p.sel_logit = sel_logit;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.scale = h->scale;
+  p.z = h->z;
+  p.z_stride = h->z_stride;
+  p.status = h->status;
+  const dim3 grid(h->batch * h->h_q);
+  const cudaError_t e = (h->d == 64)
+      ? launch(h, topn_kernel<64>, grid, dim3(kTopnThreads), kTopnSmemBytes, true, p)
+      : launch(h, topn_kernel<128>, grid, dim3(kTopnThreads), kTopnSmemBytes, true, p);
+  return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
@@ -173,14 +266,13 @@ int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
   p.sel_idx = sel_idx;
   p.sel_logit = sel_logit;
   p.status = h->status;
-  select_kernel<<<h->batch * h->h_q, kSelThreads, sizeof(SelectSmem), h->stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
-  ++h->launches;
-  return SAGA_OK;
+  const cudaError_t e = launch(h, select_kernel, dim3(h->batch * h->h_q), dim3(kSelThreads),
+                               sizeof(SelectSmem), false, p);
+  return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 int launch_gather(saga_ctx* h, const int32_t* sel_idx, const float* sel_logit,
-                  const int32_t* seq_lens, const void* v_cache, int N, void* out) {
+                  const int32_t* seq_lens, const void* v_cache, int N, void* out, bool pdl) {
   GatherParams p;
   p.sel_idx = sel_idx;
   p.sel_logit = sel_logit;
@@ -198,13 +290,10 @@ int launch_gather(saga_ctx* h, const int32_t* sel_idx, const float* sel_logit,
   p.status = h->status;
   const int slots = N < h->max_seq_len ? N : h->max_seq_len;
   const dim3 grid(h->batch * h->h_q, (slots + kGatherRows - 1) / kGatherRows);
-  if (h->d == 64)
-    gather_kernel<64><<<grid, kGatherThreads, 0, h->stream>>>(p);
-  else
-    gather_kernel<128><<<grid, kGatherThreads, 0, h->stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
-  ++h->launches;
-  return SAGA_OK;
+  const cudaError_t e = (h->d == 64)
+      ? launch(h, gather_kernel<64>, grid, dim3(kGatherThreads), 0, pdl, p)
+      : launch(h, gather_kernel<128>, grid, dim3(kGatherThreads), 0, pdl, p);
+  return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 int check_heads(saga_ctx* h, int h_q, int h_k, int h_v, int d) {
@@ -234,6 +323,14 @@ struct DeviceGuard {   // run a call on the handle's device, restore the caller'
   }
 };
 
+// The candidate path (threshold -> score pass with fused compare -> selection
+// from candidates -> gather) needs the candidate lists and a selection small
+// enough for them; otherwise every score goes through the score workspace.
+bool use_candidates(const saga_ctx* h, int N) {
+  return h->cand_key != nullptr && N <= kTopnCap / 4 &&
+         (N < h->max_seq_len || h->max_seq_len <= kTopnCap);
+}
+
 int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
                 const int32_t* seq_lens, int N, void* out, int32_t* sel_idx, float* sel_logit) {
   if (!q || !k_cache || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
@@ -242,18 +339,23 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   if (!dg.ok) return SAGA_ERR_CUDA;
   const bool prof = h->prof && h->prof_n < h->prof_max;
   cudaEvent_t* ev = prof ? &h->ev[3 * h->prof_n] : nullptr;
-  if (prof && record_event(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
-  int rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true);
-  if (rc) return rc;
-  if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
   // The selection goes to the caller's arrays when given, else to the workspace
   // (row stride N either way).
   int32_t* si = sel_idx ? sel_idx : h->sel_idx;
   float* sl = sel_logit ? sel_logit : h->sel_logit;
-  rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl);
-  if (rc) return rc;
-  rc = launch_gather(h, si, sl, seq_lens, v_cache, N, out);
-  if (rc) return rc;
+  if (prof && record_event(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+  int rc;
+  if (use_candidates(h, N)) {
+    if ((rc = launch_threshold(h, q, k_cache, seq_lens, N))) return rc;
+    if ((rc = launch_score(h, q, k_cache, seq_lens, nullptr, 0, false))) return rc;
+    if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    if ((rc = launch_topn(h, q, k_cache, seq_lens, N, si, sl))) return rc;
+  } else {
+    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true))) return rc;
+    if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    if ((rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl))) return rc;
+  }
+  if ((rc = launch_gather(h, si, sl, seq_lens, v_cache, N, out, true))) return rc;
   if (prof) {
     if (record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     ++h->prof_n;
@@ -321,9 +423,13 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->max_chunks = (slots + kGatherRows - 1) / kGatherRows;
   const size_t part_bytes = rows * h->max_chunks * (head_dim + 2) * sizeof(float);
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  // candidate lists: 8 bytes x kTopnCap per row, kept only when they stay modest
+  const size_t cand_bytes = rows * static_cast<size_t>(kTopnCap) * 4;
+  const bool keep_cand = 2 * cand_bytes <= (size_t(1) << 30);
   const size_t total = al(z_bytes) + 2 * al(stat_bytes) + 2 * al(sel_bytes) + al(256) +
                        2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4) +
-                       al(part_bytes) + al(stat_bytes);
+                       al(part_bytes) + al(stat_bytes) + 2 * al(stat_bytes) +
+                       (keep_cand ? 2 * al(cand_bytes) : 0);
   if (cudaMalloc(&h->ws, total) != cudaSuccess) { delete h; return SAGA_ERR_CUDA; }
   uint8_t* w = static_cast<uint8_t*>(h->ws);
   h->z = reinterpret_cast<float*>(w); w += al(z_bytes);
@@ -336,9 +442,17 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->out_stage = reinterpret_cast<__nv_bfloat16*>(w); w += al(qo_bytes);
   h->lens_stage = reinterpret_cast<int32_t*>(w); w += al(static_cast<size_t>(max_batch) * 4);
   h->partial = reinterpret_cast<float*>(w); w += al(part_bytes);
-  h->counter = reinterpret_cast<uint32_t*>(w);
+  h->counter = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
+  h->t_lo = reinterpret_cast<float*>(w); w += al(stat_bytes);
+  h->cand_count = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
+  if (keep_cand) {
+    h->cand_key = reinterpret_cast<uint32_t*>(w); w += al(cand_bytes);
+    h->cand_pos = reinterpret_cast<int32_t*>(w);
+  }
+  h->scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
   if (cudaMemset(h->stat_min, 0xFF, stat_bytes) != cudaSuccess ||
       cudaMemset(h->counter, 0x00, stat_bytes) != cudaSuccess ||
+      cudaMemset(h->cand_count, 0x00, stat_bytes) != cudaSuccess ||
       cudaMemset(h->stat_max, 0x00, stat_bytes) != cudaSuccess ||
       cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->ws);
@@ -432,7 +546,7 @@ int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
   if (cudaMemsetAsync(h->counter, 0, static_cast<size_t>(h->batch) * h->h_q * sizeof(uint32_t),
                       h->stream) != cudaSuccess)
     return SAGA_ERR_CUDA;
-  return launch_gather(h, sel_idx, sel_logit, seq_lens, v_cache, N, out);
+  return launch_gather(h, sel_idx, sel_logit, seq_lens, v_cache, N, out, false);
 }
 
 int saga_decode_status(saga_handle h, int* device_status) {
@@ -460,16 +574,19 @@ int saga_decode_profile(saga_handle h, int enable, int max_calls) {
   if (!h || (enable && max_calls < 1)) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
-  for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
-  h->ev.clear();
-  h->prof = false;
-  h->prof_n = 0;
-  h->prof_max = 0;
-  if (!enable) return SAGA_OK;
-  h->ev.resize(3 * static_cast<size_t>(max_calls));
-  for (auto& e : h->ev)
-    if (cudaEventCreate(&e) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (!enable) {                 // stop recording; keep the events (a captured graph may use them)
+    h->prof = false;
+    return SAGA_OK;
+  }
+  if (h->ev.size() < 3 * static_cast<size_t>(max_calls)) {
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    h->ev.assign(3 * static_cast<size_t>(max_calls), nullptr);
+    for (auto& e : h->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return SAGA_ERR_CUDA;
+  }
   h->prof_max = max_calls;
+  h->prof_n = 0;
   h->prof = true;
   return SAGA_OK;
 }

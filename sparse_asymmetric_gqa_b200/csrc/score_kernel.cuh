@@ -32,7 +32,13 @@ constexpr int kMaxBatch = 1024;
 
 struct ScoreParams {
   const int32_t* seq_lens;   // [B]
-  float* z;                  // [B*h_q][z_stride]
+  float* z;                  // [B*h_q][z_stride] (score-row mode)
+  // candidate mode: scores >= t_lo[row] are appended to the row's list
+  const float* t_lo;         // [B*h_q]
+  uint32_t* cand_count;      // [B*h_q], zero on entry
+  uint32_t* cand_key;        // [B*h_q][cand_cap] ordered keys
+  int32_t* cand_pos;         // [B*h_q][cand_cap] positions
+  int cand_cap;
   uint32_t* stat_min;        // [B*h_q] ordered keys, or nullptr
   uint32_t* stat_max;
   int* status;
@@ -97,7 +103,12 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
   atomicOr(status, 0x2 /* SAGA_STATUS_TIMEOUT */);
 }
 
-template <int D, int NPAD>
+// kCand = false: every score is stored to z (row stride z_stride) and per-row
+// min/max keys are kept.  kCand = true: nothing is stored but the candidates
+// of the selector, every (key, position) whose score is >= t_lo of its row,
+// appended with one atomic per warp and head; the kernel then waits for the
+// preceding kernel (which writes t_lo) before its epilogue reads t_lo.
+template <int D, int NPAD, bool kCand>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_kernel(const __grid_constant__ CUtensorMap tmap_k,
              const __grid_constant__ CUtensorMap tmap_q, const ScoreParams p) {
@@ -123,6 +134,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
   if (warp == 0) {
     if (lane == 0) {
+      if (kCand) pdl_launch_dependents();
       for (int s = 0; s < S::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
       for (int i = 0; i < 2; ++i) { mbar_init(accf_bar(i), 1); mbar_init(acce_bar(i), kEpiWarps); }
       mbar_init(drain_bar, 1);
@@ -260,6 +272,10 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         rmax[i] = 0u;
       }
     };
+    float tl[H];
+#pragma unroll
+    for (int e = 0; e < H; ++e) tl[e] = INFINITY;
+    if (kCand) pdl_wait();                      // t_lo comes from the preceding kernel
     if (n_tiles > 0) {
       TileCursor c;
       c.seek(u0, unit_off, lens, p.B, p.h_k);
@@ -284,10 +300,48 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         __syncwarp();
         if (lane == 0) mbar_arrive(acce_bar(buf));
 
-        if (c.b != seg_b || c.kh != seg_kh) { flush(); seg_b = c.b; seg_kh = c.kh; }
+        const int row0 = c.b * p.h_q + c.kh * p.g + h0;     // z row of head h0
+        if (c.b != seg_b || c.kh != seg_kh) {
+          if (!kCand) flush();
+          seg_b = c.b;
+          seg_kh = c.kh;
+          if (kCand) {
+#pragma unroll
+            for (int e = 0; e < H; ++e) tl[e] = (h0 + e < p.g) ? p.t_lo[row0 + e] : INFINITY;
+          }
+        }
         const int pos = c.t * kTileM + quad * 32 + lane;
-        if (pos < c.Lb) {
-          float* zrow = p.z + static_cast<long long>(c.b * p.h_q + c.kh * p.g + h0) * p.z_stride + pos;
+        const bool valid = pos < c.Lb;
+        if (kCand) {
+          const uint32_t lt = (1u << lane) - 1u;
+          float zz[H];
+          uint32_t m[H];
+          uint32_t my_m = 0u;
+#pragma unroll
+          for (int e = 0; e < H; ++e) {
+            // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
+            zz[e] = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
+            m[e] = __ballot_sync(0xffffffffu, valid && h0 + e < p.g && zz[e] >= tl[e]);
+            if (lane == e) my_m = m[e];
+          }
+          // lane e reserves the slots of head e, so the H atomics are in flight together
+          uint32_t my_base = 0u;
+          if (lane < H && my_m != 0u)
+            my_base = atomicAdd(p.cand_count + row0 + lane, static_cast<uint32_t>(__popc(my_m)));
+#pragma unroll
+          for (int e = 0; e < H; ++e) {
+            const uint32_t base = __shfl_sync(0xffffffffu, my_base, e);
+            if ((m[e] >> lane) & 1u) {
+              const uint32_t slot = base + __popc(m[e] & lt);
+              if (slot < static_cast<uint32_t>(p.cand_cap)) {
+                const long long o = static_cast<long long>(row0 + e) * p.cand_cap + slot;
+                p.cand_key[o] = ordered_key(zz[e]);
+                p.cand_pos[o] = pos;
+              }
+            }
+          }
+        } else if (valid) {
+          float* zrow = p.z + static_cast<long long>(row0) * p.z_stride + pos;
 #pragma unroll
           for (int e = 0; e < H; ++e) {
             if (h0 + e < p.g) {
@@ -302,7 +356,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         c.next(unit_off, lens, p.B, p.h_k);
       }
-      flush();
+      if (!kCand) flush();
     }
   }
 
