@@ -73,9 +73,9 @@ gather_kernel(const GatherParams p) {
   float z = -INFINITY;
   if (r < n_slots) {
     const long long o = static_cast<long long>(bj) * p.N + r;
-    id = p.sel_idx[o];
+    id = __ldcg(p.sel_idx + o);
     if (id >= L) { atomicOr(p.status, 0x4 /* SAGA_STATUS_BAD_INDEX */); id = -1; }
-    if (id >= 0) z = p.sel_logit[o];
+    if (id >= 0) z = __ldcg(p.sel_logit + o);
   }
   float m = z;
   for (int s = 16; s; s >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, s));

@@ -24,8 +24,8 @@
 #include "score_kernel.cuh"
 #include "select_kernel.cuh"
 #include "gather_kernel.cuh"
-#include "threshold_kernel.cuh"
 #include "topn_kernel.cuh"
+#include "bound_kernel.cuh"
 
 using namespace saga;
 
@@ -87,10 +87,10 @@ struct saga_ctx {
   __nv_bfloat16* out_stage = nullptr;
   int32_t* lens_stage = nullptr;
   float scale = 0.0f;             // 1/sqrt(d) rounded to fp32
-  float* t_lo = nullptr;          // candidate thresholds [rows]
-  uint32_t* cand_count = nullptr; // candidates appended per row [rows]
-  uint32_t* cand_key = nullptr;   // candidate lists [rows][kTopnCap] (null: lists not kept)
-  int32_t* cand_pos = nullptr;
+  uint32_t* cand_mask = nullptr;  // candidate chunk masks [rows][mask_stride]
+  long long mask_stride = 0;      // z_stride / 32
+  float* samp = nullptr;          // sampled scores [rows][kSampleSize]
+  float* t_lo = nullptr;          // candidate bounds [rows]
   float* partial = nullptr;       // gather partials [rows][max_chunks][d + 2]
   uint32_t* counter = nullptr;    // gather merge counters [rows]
   int max_chunks = 0;
@@ -132,47 +132,52 @@ int set_smem_attrs_once() {
   return rc;
 }
 
-// Launch on the handle's stream; with `pdl` the kernel may start before the
+// Launch on the handle's stream.  kPdl: the kernel may start before the
 // previous kernel in the stream has finished (it waits in-kernel before it
-// reads that kernel's results: programmatic dependent launch).
+// reads that kernel's results: programmatic dependent launch).  kCoop: all
+// CTAs are resident at once (cooperative launch; the kernel synchronises
+// across the grid).
+enum LaunchMode { kPlain = 0, kPdl = 1, kCoop = 2 };
 template <typename... KArgs, typename... Args>
 cudaError_t launch(saga_ctx* h, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                   bool pdl, Args&&... args) {
+                   int mode, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = h->stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (mode == kPdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = (mode == kPlain) ? 0 : 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e == cudaSuccess) ++h->launches;
   return e;
 }
 
-// Score pass.  z == nullptr: candidate mode (thresholds from h->t_lo, lists in
-// the workspace, launched as a dependent of the threshold kernel); otherwise
-// every score goes to z.
+// Score pass.  cand: candidate mode (bounds from h->t_lo, chunk masks and
+// candidate keys in the workspace; a programmatic dependent of the bound
+// kernel); otherwise every score goes to z.
 int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
-                 float* z, long long z_stride, bool stats) {
+                 float* z, long long z_stride, bool stats, bool cand = false) {
   CUtensorMap mk, mq;
   const uint64_t k_rows = static_cast<uint64_t>(h->batch) * h->h_k * h->max_seq_len;
   const uint64_t q_rows = static_cast<uint64_t>(h->batch) * h->h_q;
   if (!encode_bf16_2d(&mk, k_cache, k_rows, h->d, kTileM)) return SAGA_ERR_CUDA;
   if (!encode_bf16_2d(&mq, q, q_rows, h->d, h->npad)) return SAGA_ERR_CUDA;
-  const bool cand = (z == nullptr);
   ScoreParams p;
   std::memset(&p, 0, sizeof(p));
   p.seq_lens = seq_lens;
   p.z = z;
+  p.cand_mask = h->cand_mask;
+  p.mask_stride = h->mask_stride;
   p.t_lo = h->t_lo;
-  p.cand_count = h->cand_count;
-  p.cand_key = h->cand_key;
-  p.cand_pos = h->cand_pos;
-  p.cand_cap = kTopnCap;
   p.stat_min = (stats && !cand) ? h->stat_min : nullptr;
   p.stat_max = (stats && !cand) ? h->stat_max : nullptr;
   p.status = h->status;
@@ -190,18 +195,19 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
 #define SAGA_CASE(D, NP)                                                                       \
   if (h->d == D && h->npad == NP)                                                              \
     e = cand ? launch(h, score_kernel<D, NP, true>, dim3(grid), dim3(kScoreThreads),           \
-                      ScoreShape<D, NP>::kSmemBytes, true, mk, mq, p)                          \
+                      ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p)                          \
              : launch(h, score_kernel<D, NP, false>, dim3(grid), dim3(kScoreThreads),          \
-                      ScoreShape<D, NP>::kSmemBytes, false, mk, mq, p);
+                      ScoreShape<D, NP>::kSmemBytes, kPlain, mk, mq, p);
   SAGA_CASE(64, 16) SAGA_CASE(64, 32) SAGA_CASE(64, 48) SAGA_CASE(64, 64)
   SAGA_CASE(128, 16) SAGA_CASE(128, 32) SAGA_CASE(128, 48) SAGA_CASE(128, 64)
 #undef SAGA_CASE
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
-int launch_threshold(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
-                     int N) {
-  ThresholdParams p;
+// Candidate bounds: the sample kernel (after the previous kernel in the stream)
+// and the bound kernel (a programmatic dependent of it).
+int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens, int N) {
+  BoundParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   p.seq_lens = seq_lens;
@@ -212,21 +218,24 @@ int launch_threshold(saga_ctx* h, const void* q, const void* k_cache, const int3
   p.N = N;
   p.cand_cap = kTopnCap;
   p.scale = h->scale;
+  p.samp = h->samp;
   p.t_lo = h->t_lo;
-  const dim3 grid(h->batch * h->h_q);
-  const cudaError_t e = (h->d == 64)
-      ? launch(h, threshold_kernel<64>, grid, dim3(kThrThreads), 0, false, p)
-      : launch(h, threshold_kernel<128>, grid, dim3(kThrThreads), 0, false, p);
+  const dim3 sgrid(h->batch * h->h_k, kSampleParts);
+  const size_t smem = static_cast<size_t>(h->g) * h->d * sizeof(float);
+  cudaError_t e = (h->d == 64)
+      ? launch(h, sample_kernel<64>, sgrid, dim3(kSampleThreads), smem, kPlain, p)
+      : launch(h, sample_kernel<128>, sgrid, dim3(kSampleThreads), smem, kPlain, p);
+  if (e == cudaSuccess) e = launch(h, bound_kernel, dim3(h->batch * h->h_q), dim3(32), 0, kPdl, p);
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens, int N,
                 int32_t* sel_idx, float* sel_logit) {
   TopnParams p;
-  p.cand_key = h->cand_key;
-  p.cand_pos = h->cand_pos;
-  p.cand_count = h->cand_count;
-  p.cand_cap = kTopnCap;
+  p.cand_mask = h->cand_mask;
+  p.mask_stride = h->mask_stride;
+  p.zkey = reinterpret_cast<uint32_t*>(h->z);
+  p.z_stride = h->z_stride;
   p.gather_count = h->counter;
   p.seq_lens = seq_lens;
   p.h_q = h->h_q;
@@ -239,13 +248,11 @@ int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const int32_t* 
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   p.scale = h->scale;
-  p.z = h->z;
-  p.z_stride = h->z_stride;
   p.status = h->status;
   const dim3 grid(h->batch * h->h_q);
   const cudaError_t e = (h->d == 64)
-      ? launch(h, topn_kernel<64>, grid, dim3(kTopnThreads), kTopnSmemBytes, true, p)
-      : launch(h, topn_kernel<128>, grid, dim3(kTopnThreads), kTopnSmemBytes, true, p);
+      ? launch(h, topn_kernel<64>, grid, dim3(kTopnThreads), kTopnSmemBytes, kPdl, p)
+      : launch(h, topn_kernel<128>, grid, dim3(kTopnThreads), kTopnSmemBytes, kPdl, p);
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
@@ -267,7 +274,7 @@ int launch_select(saga_ctx* h, const float* z, long long z_stride, bool stats,
   p.sel_logit = sel_logit;
   p.status = h->status;
   const cudaError_t e = launch(h, select_kernel, dim3(h->batch * h->h_q), dim3(kSelThreads),
-                               sizeof(SelectSmem), false, p);
+                               sizeof(SelectSmem), kPlain, p);
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
@@ -291,8 +298,8 @@ int launch_gather(saga_ctx* h, const int32_t* sel_idx, const float* sel_logit,
   const int slots = N < h->max_seq_len ? N : h->max_seq_len;
   const dim3 grid(h->batch * h->h_q, (slots + kGatherRows - 1) / kGatherRows);
   const cudaError_t e = (h->d == 64)
-      ? launch(h, gather_kernel<64>, grid, dim3(kGatherThreads), 0, pdl, p)
-      : launch(h, gather_kernel<128>, grid, dim3(kGatherThreads), 0, pdl, p);
+      ? launch(h, gather_kernel<64>, grid, dim3(kGatherThreads), 0, pdl ? kPdl : kPlain, p)
+      : launch(h, gather_kernel<128>, grid, dim3(kGatherThreads), 0, pdl ? kPdl : kPlain, p);
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
@@ -323,11 +330,11 @@ struct DeviceGuard {   // run a call on the handle's device, restore the caller'
   }
 };
 
-// The candidate path (threshold -> score pass with fused compare -> selection
-// from candidates -> gather) needs the candidate lists and a selection small
+// The candidate path (sampled bounds -> score pass with fused compare ->
+// selection from candidates -> gather) needs the candidate lists and a selection small
 // enough for them; otherwise every score goes through the score workspace.
 bool use_candidates(const saga_ctx* h, int N) {
-  return h->cand_key != nullptr && N <= kTopnCap / 4 &&
+  return h->cand_mask != nullptr && N <= kTopnCap / 4 &&
          (N < h->max_seq_len || h->max_seq_len <= kTopnCap);
 }
 
@@ -346,8 +353,8 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   if (prof && record_event(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
   int rc;
   if (use_candidates(h, N)) {
-    if ((rc = launch_threshold(h, q, k_cache, seq_lens, N))) return rc;
-    if ((rc = launch_score(h, q, k_cache, seq_lens, nullptr, 0, false))) return rc;
+    if ((rc = launch_bounds(h, q, k_cache, seq_lens, N))) return rc;
+    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true))) return rc;
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     if ((rc = launch_topn(h, q, k_cache, seq_lens, N, si, sl))) return rc;
   } else {
@@ -423,13 +430,13 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->max_chunks = (slots + kGatherRows - 1) / kGatherRows;
   const size_t part_bytes = rows * h->max_chunks * (head_dim + 2) * sizeof(float);
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  // candidate lists: 8 bytes x kTopnCap per row, kept only when they stay modest
-  const size_t cand_bytes = rows * static_cast<size_t>(kTopnCap) * 4;
-  const bool keep_cand = 2 * cand_bytes <= (size_t(1) << 30);
+  // candidate path: chunk masks (the keys reuse z), sampled scores, bounds
+  h->mask_stride = h->z_stride / 32;
+  const size_t mask_bytes = rows * static_cast<size_t>(h->mask_stride) * 4;
+  const size_t samp_bytes = rows * static_cast<size_t>(kSampleSize) * 4;
   const size_t total = al(z_bytes) + 2 * al(stat_bytes) + 2 * al(sel_bytes) + al(256) +
                        2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4) +
-                       al(part_bytes) + al(stat_bytes) + 2 * al(stat_bytes) +
-                       (keep_cand ? 2 * al(cand_bytes) : 0);
+                       al(part_bytes) + 2 * al(stat_bytes) + al(mask_bytes) + al(samp_bytes);
   if (cudaMalloc(&h->ws, total) != cudaSuccess) { delete h; return SAGA_ERR_CUDA; }
   uint8_t* w = static_cast<uint8_t*>(h->ws);
   h->z = reinterpret_cast<float*>(w); w += al(z_bytes);
@@ -443,16 +450,12 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->lens_stage = reinterpret_cast<int32_t*>(w); w += al(static_cast<size_t>(max_batch) * 4);
   h->partial = reinterpret_cast<float*>(w); w += al(part_bytes);
   h->counter = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
-  h->t_lo = reinterpret_cast<float*>(w); w += al(stat_bytes);
-  h->cand_count = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
-  if (keep_cand) {
-    h->cand_key = reinterpret_cast<uint32_t*>(w); w += al(cand_bytes);
-    h->cand_pos = reinterpret_cast<int32_t*>(w);
-  }
+  h->cand_mask = reinterpret_cast<uint32_t*>(w); w += al(mask_bytes);
+  h->samp = reinterpret_cast<float*>(w); w += al(samp_bytes);
+  h->t_lo = reinterpret_cast<float*>(w);
   h->scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
   if (cudaMemset(h->stat_min, 0xFF, stat_bytes) != cudaSuccess ||
       cudaMemset(h->counter, 0x00, stat_bytes) != cudaSuccess ||
-      cudaMemset(h->cand_count, 0x00, stat_bytes) != cudaSuccess ||
       cudaMemset(h->stat_max, 0x00, stat_bytes) != cudaSuccess ||
       cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->ws);

@@ -13,11 +13,15 @@
 //   * warp 0 streams K tiles (and the group's q rows) into a ring of shared
 //     memory stages with TMA (128-byte swizzle, L2 evict-first for K);
 //   * warp 1 issues tcgen05.mma (M = 128 positions, N = g padded to 16k,
-//     K = 16 per instruction) into a double-buffered TMEM accumulator;
-//   * warps 2-9 read the accumulator back with tcgen05.ld (thread = position,
-//     registers = heads; two warps per TMEM lane quarter, each taking half of
-//     the heads), scale, store z row-wise (coalesced per head) and keep
-//     per-(b, j) min/max statistics in registers for the selector.
+//     K = 16 per instruction) into a ring of TMEM accumulators that fills all
+//     512 columns (32 tiles for g <= 16), so the K stream runs on while the
+//     epilogue waits for the sampled bounds;
+//   * warps 2-9 read the accumulators back with tcgen05.ld (thread = position,
+//     registers = heads), two warps per TMEM lane quarter: for groups of up to
+//     32 heads the two warp sets take alternate tiles (so two tiles are read
+//     back at once), for larger groups each takes half of the heads.  They
+//     scale, and either store z row-wise (coalesced per head) with per-(b, j)
+//     min/max statistics, or append the candidates of the selector.
 #pragma once
 
 #include <cuda.h>
@@ -32,13 +36,11 @@ constexpr int kMaxBatch = 1024;
 
 struct ScoreParams {
   const int32_t* seq_lens;   // [B]
-  float* z;                  // [B*h_q][z_stride] (score-row mode)
-  // candidate mode: scores >= t_lo[row] are appended to the row's list
-  const float* t_lo;         // [B*h_q]
-  uint32_t* cand_count;      // [B*h_q], zero on entry
-  uint32_t* cand_key;        // [B*h_q][cand_cap] ordered keys
-  int32_t* cand_pos;         // [B*h_q][cand_cap] positions
-  int cand_cap;
+  float* z;                  // [B*h_q][z_stride]: scores, or candidate keys in candidate mode
+  // candidate mode: the scores >= t_lo[row] of each 32-position chunk of a row
+  uint32_t* cand_mask;       // [B*h_q][mask_stride]: bit i of word c = position 32c + i passed
+  long long mask_stride;
+  const float* t_lo;         // [B*h_q] candidate bounds, written by the preceding kernel
   uint32_t* stat_min;        // [B*h_q] ordered keys, or nullptr
   uint32_t* stat_max;
   int* status;
@@ -57,9 +59,15 @@ struct ScoreShape {
   static constexpr int kStageBytes = kParts * (kAPart + kBPart);
   static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesRaw < 8 ? kStagesRaw : 8;
-  static constexpr int kTmemCols = (2 * NPAD <= 32) ? 32 : ((2 * NPAD <= 64) ? 64 : 128);
-  static constexpr int kAccStride = kTmemCols / 2;      // column offset of accumulator 1
-  static constexpr int kNumBars = 2 * kStages + 5;      // full, empty, accf[2], acce[2], drain
+  static constexpr int kAccStride = NPAD <= 16 ? 16 : NPAD <= 32 ? 32 : 64;   // columns per accumulator
+  static constexpr int kTmemCols = 512;                                        // all of TMEM
+  static constexpr int kAccBufs = kTmemCols / kAccStride;                      // 32, 16 or 8
+  // full, empty, accf[kAccBufs], acce[kAccBufs], drain
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
+  // Epilogue split: tile groups (alternate tiles) for up to 32 heads, else head halves.
+  static constexpr int kTileGroups = NPAD <= 32 ? 2 : 1;
+  static constexpr int kEpiHeads = NPAD * kTileGroups / 2;   // heads per epilogue warp
+  // bars, TMEM slot + abort flag, lens, unit_off
   static constexpr int kCtrlBytes = kNumBars * 8 + 16 + 2 * (kMaxBatch + 1) * 4;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kCtrlBytes;
   static_assert(kStages >= 2, "stages");
@@ -104,10 +112,14 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 }
 
 // kCand = false: every score is stored to z (row stride z_stride) and per-row
-// min/max keys are kept.  kCand = true: nothing is stored but the candidates
-// of the selector, every (key, position) whose score is >= t_lo of its row,
-// appended with one atomic per warp and head; the kernel then waits for the
-// preceding kernel (which writes t_lo) before its epilogue reads t_lo.
+// min/max keys are kept.
+// kCand = true (launched as a programmatic dependent of the bound kernel): only
+// the candidates of the selector are stored.  The producer and MMA warps start
+// streaming at once; the epilogue first waits for the bounds t_lo.  Then, for
+// each 32-position chunk c of a row, the mask of positions with score >= t_lo
+// goes to cand_mask[row][c] and their order-preserving keys, in position
+// order, to the row's z slots [32c, 32c + popcount).  No atomics on the data
+// path: every chunk has its own slots.
 template <int D, int NPAD, bool kCand>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -129,14 +141,17 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S::kStages + s); };
   auto accf_bar = [&](int i) { return bar0 + 8u * (2 * S::kStages + i); };
-  auto acce_bar = [&](int i) { return bar0 + 8u * (2 * S::kStages + 2 + i); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * S::kStages + 4);
+  auto acce_bar = [&](int i) { return bar0 + 8u * (2 * S::kStages + S::kAccBufs + i); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * S::kStages + 2 * S::kAccBufs);
 
   if (warp == 0) {
     if (lane == 0) {
       if (kCand) pdl_launch_dependents();
       for (int s = 0; s < S::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-      for (int i = 0; i < 2; ++i) { mbar_init(accf_bar(i), 1); mbar_init(acce_bar(i), kEpiWarps); }
+      for (int i = 0; i < S::kAccBufs; ++i) {
+        mbar_init(accf_bar(i), 1);
+        mbar_init(acce_bar(i), kEpiWarps / S::kTileGroups);   // warps that read each tile
+      }
       mbar_init(drain_bar, 1);
       *abort_flag = 0;
       fence_mbar_init();
@@ -177,22 +192,25 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const long long u0 = total * blockIdx.x / gridDim.x;
   const long long u1 = total * (blockIdx.x + 1) / gridDim.x;
   const int n_tiles = static_cast<int>(u1 - u0);
+  const int n_items = n_tiles;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0 && n_items > 0) {
       const uint64_t pol_k = policy_evict_first();
       const uint64_t pol_q = policy_evict_last();
       TileCursor c;
       c.seek(u0, unit_off, lens, p.B, p.h_k);
       int i = 0;
-      for (; i < n_tiles; ++i) {
+      for (; i < n_items; ++i) {
         const int s = i % S::kStages;
         const uint32_t ph = (i / S::kStages) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag)) { raise_abort(abort_flag, p.status); break; }
+        const int b = c.b, kh = c.kh, t = c.t;
+        c.next(unit_off, lens, p.B, p.h_k);
         mbar_arrive_expect_tx(full_bar(s), S::kStageBytes);
-        const int row = (c.b * p.h_k + c.kh) * p.L_max + c.t * kTileM;
-        const int qrow = c.b * p.h_q + c.kh * p.g;
+        const int row = (b * p.h_k + kh) * p.L_max + t * kTileM;
+        const int qrow = b * p.h_q + kh * p.g;
         const uint32_t a = smem_addr(stages + s * S::kStageBytes);
         const uint32_t bq = a + S::kParts * S::kAPart;
 #pragma unroll
@@ -201,7 +219,6 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
         for (int part = 0; part < S::kParts; ++part)
           tma_load_2d(bq + part * S::kBPart, &tmap_q, part * 64, qrow, full_bar(s), pol_q);
-        c.next(unit_off, lens, p.B, p.h_k);
       }
       // Let every load this thread issued land before the CTA can exit.
       const int first = i > S::kStages ? i - S::kStages : 0;
@@ -212,14 +229,14 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0 && n_items > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTileM, NPAD);
       int i = 0;
-      for (; i < n_tiles; ++i) {
+      for (; i < n_items; ++i) {
         const int s = i % S::kStages;
         const uint32_t ph = (i / S::kStages) & 1;
-        const int buf = i & 1;
-        const uint32_t aph = (i >> 1) & 1;
+        const int buf = i % S::kAccBufs;
+        const uint32_t aph = (i / S::kAccBufs) & 1;
         if (!mbar_wait(acce_bar(buf), aph ^ 1, abort_flag)) { raise_abort(abort_flag, p.status); break; }
         if (!mbar_wait(full_bar(s), ph, abort_flag)) { raise_abort(abort_flag, p.status); break; }
         tc_fence_after();
@@ -244,102 +261,101 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Warp w reads TMEM lane quarter w % 4 (the hardware rule) and heads
-    // [half * H, half * H + H) of the group, half = (w - 2) / 4.
-    constexpr int H = NPAD / 2;
+    // Warp w reads TMEM lane quarter w % 4 (the hardware rule); its set
+    // (w - 2) / 4 takes the items of that parity (two tile groups) or the
+    // heads [set * H, set * H + H) of every item (one tile group).
+    constexpr int H = S::kEpiHeads;
+    constexpr int TG = S::kTileGroups;
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int h0 = half * H;
+    const int set = (warp - 2) >> 2;
+    const int h0 = (TG == 1) ? set * H : 0;
     const uint64_t pol_z = policy_evict_last();
+    bool alive = true;
+    // Item i's accumulator, heads h0 .. h0 + H - 1 of this lane's position.
+    auto read_acc = [&](int i, float* acc) -> bool {
+      const int buf = i % S::kAccBufs;
+      const uint32_t aph = (i / S::kAccBufs) & 1;
+      // every lane waits; the decision to go on is taken warp-uniformly
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(accf_bar(buf), aph, abort_flag));
+      if (!ok) { if (lane == 0) raise_abort(abort_flag, p.status); return false; }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < H / 8; ++cc) {
+        float v[8];
+        tmem_ld_8(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * S::kAccStride +
+                      h0 + cc * 8, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[cc * 8 + e] = v[e];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(buf));
+      return true;
+    };
+    if (kCand) pdl_wait();                        // t_lo comes from the preceding kernel
+
     uint32_t rmin[H], rmax[H];
 #pragma unroll
-    for (int i = 0; i < H; ++i) { rmin[i] = 0xFFFFFFFFu; rmax[i] = 0u; }
+    for (int e = 0; e < H; ++e) { rmin[e] = 0xFFFFFFFFu; rmax[e] = 0u; }
     int seg_b = -1, seg_kh = -1;
     auto flush = [&]() {
 #pragma unroll
-      for (int i = 0; i < H; ++i) {
-        const int h = h0 + i;
+      for (int e = 0; e < H; ++e) {
+        const int h = h0 + e;
         if (h < p.g) {
-          const uint32_t kmin = __reduce_min_sync(0xffffffffu, rmin[i]);
-          const uint32_t kmax = __reduce_max_sync(0xffffffffu, rmax[i]);
+          const uint32_t kmin = __reduce_min_sync(0xffffffffu, rmin[e]);
+          const uint32_t kmax = __reduce_max_sync(0xffffffffu, rmax[e]);
           if (lane == 0 && seg_b >= 0 && p.stat_min != nullptr && kmin <= kmax) {
             const int bj = seg_b * p.h_q + seg_kh * p.g + h;
             atomicMin(p.stat_min + bj, kmin);
             atomicMax(p.stat_max + bj, kmax);
           }
         }
-        rmin[i] = 0xFFFFFFFFu;
-        rmax[i] = 0u;
+        rmin[e] = 0xFFFFFFFFu;
+        rmax[e] = 0u;
       }
     };
     float tl[H];
 #pragma unroll
     for (int e = 0; e < H; ++e) tl[e] = INFINITY;
-    if (kCand) pdl_wait();                      // t_lo comes from the preceding kernel
     if (n_tiles > 0) {
       TileCursor c;
       c.seek(u0, unit_off, lens, p.B, p.h_k);
-      for (int i = 0; i < n_tiles; ++i) {
-        const int buf = i & 1;
-        const uint32_t aph = (i >> 1) & 1;
-        // every lane waits; the decision to go on is taken warp-uniformly
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(accf_bar(buf), aph, abort_flag));
-        if (!ok) { if (lane == 0) raise_abort(abort_flag, p.status); break; }
-        tc_fence_after();
-        float acc[H];
-#pragma unroll
-        for (int cc = 0; cc < H / 8; ++cc) {
-          float v[8];
-          tmem_ld_8(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + buf * S::kAccStride +
-                        h0 + cc * 8, v);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[cc * 8 + e] = v[e];
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acce_bar(buf));
-
-        const int row0 = c.b * p.h_q + c.kh * p.g + h0;     // z row of head h0
-        if (c.b != seg_b || c.kh != seg_kh) {
+      for (int jt = 0; jt < n_tiles; ++jt, c.next(unit_off, lens, p.B, p.h_k)) {
+        const int i = jt;                         // index in the pipeline
+        if (!alive || (TG == 2 && (i & 1) != set)) continue;
+        if (c.b != seg_b || c.kh != seg_kh) {     // a new row segment
           if (!kCand) flush();
           seg_b = c.b;
           seg_kh = c.kh;
           if (kCand) {
+            const int rowg = c.b * p.h_q + c.kh * p.g + h0;
 #pragma unroll
-            for (int e = 0; e < H; ++e) tl[e] = (h0 + e < p.g) ? p.t_lo[row0 + e] : INFINITY;
+            for (int e = 0; e < H; ++e) tl[e] = (h0 + e < p.g) ? __ldcg(p.t_lo + rowg + e) : INFINITY;
           }
         }
+        float acc[H];
+        if (!read_acc(i, acc)) { alive = false; continue; }
+        const int row0 = c.b * p.h_q + c.kh * p.g + h0;     // z row of head h0
         const int pos = c.t * kTileM + quad * 32 + lane;
         const bool valid = pos < c.Lb;
         if (kCand) {
           const uint32_t lt = (1u << lane) - 1u;
-          float zz[H];
-          uint32_t m[H];
+          const int chunk = c.t * (kTileM / 32) + quad;
+          uint32_t* kslot = reinterpret_cast<uint32_t*>(p.z) + static_cast<long long>(row0) * p.z_stride + chunk * 32;
           uint32_t my_m = 0u;
 #pragma unroll
           for (int e = 0; e < H; ++e) {
             // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
-            zz[e] = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
-            m[e] = __ballot_sync(0xffffffffu, valid && h0 + e < p.g && zz[e] >= tl[e]);
-            if (lane == e) my_m = m[e];
+            const float zz = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
+            const bool take = valid && h0 + e < p.g && zz >= tl[e];
+            const uint32_t m = __ballot_sync(0xffffffffu, take);
+            if (lane == e) my_m = m;
+            if (take) kslot[e * p.z_stride + __popc(m & lt)] = ordered_key(zz);
           }
-          // lane e reserves the slots of head e, so the H atomics are in flight together
-          uint32_t my_base = 0u;
-          if (lane < H && my_m != 0u)
-            my_base = atomicAdd(p.cand_count + row0 + lane, static_cast<uint32_t>(__popc(my_m)));
-#pragma unroll
-          for (int e = 0; e < H; ++e) {
-            const uint32_t base = __shfl_sync(0xffffffffu, my_base, e);
-            if ((m[e] >> lane) & 1u) {
-              const uint32_t slot = base + __popc(m[e] & lt);
-              if (slot < static_cast<uint32_t>(p.cand_cap)) {
-                const long long o = static_cast<long long>(row0 + e) * p.cand_cap + slot;
-                p.cand_key[o] = ordered_key(zz[e]);
-                p.cand_pos[o] = pos;
-              }
-            }
-          }
+          if (lane < H && h0 + lane < p.g && chunk * 32 < c.Lb)   // lane e: head e's mask
+            p.cand_mask[static_cast<long long>(row0 + lane) * p.mask_stride + chunk] = my_m;
         } else if (valid) {
           float* zrow = p.z + static_cast<long long>(row0) * p.z_stride + pos;
 #pragma unroll
@@ -354,7 +370,6 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
           }
         }
-        c.next(unit_off, lens, p.B, p.h_k);
       }
       if (!kCand) flush();
     }

@@ -291,7 +291,7 @@ def test_deterministic_and_host_entry_point():
     n0 = dec.launch_count()
     dec.attn_host(q_h, k, v, l_h, spec.N, o_h)
     assert dec.status() == 0
-    assert dec.launch_count() - n0 == 4   # threshold, score, top-N, gather
+    assert dec.launch_count() - n0 == 5   # sample, bound, score, top-N, gather
     assert torch.equal(o_h, a.cpu())
 
 
