@@ -229,25 +229,29 @@ int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
-int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens, int N,
-                int32_t* sel_idx, float* sel_logit) {
+// S2-S4 from the candidate lists (a programmatic dependent of the score pass).
+int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_logit, void* out) {
   TopnParams p;
   p.cand_mask = h->cand_mask;
   p.mask_stride = h->mask_stride;
   p.zkey = reinterpret_cast<uint32_t*>(h->z);
   p.z_stride = h->z_stride;
-  p.gather_count = h->counter;
   p.seq_lens = seq_lens;
   p.h_q = h->h_q;
   p.h_k = h->h_k;
   p.g = h->g;
+  p.h_v = h->h_v;
+  p.g_v = h->g_v;
   p.L_max = h->max_seq_len;
   p.N = N;
   p.sel_idx = sel_idx;
   p.sel_logit = sel_logit;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
   p.scale = h->scale;
+  p.out = static_cast<__nv_bfloat16*>(out);
   p.status = h->status;
   const dim3 grid(h->batch * h->h_q);
   const cudaError_t e = (h->d == 64)
@@ -334,7 +338,7 @@ struct DeviceGuard {   // run a call on the handle's device, restore the caller'
 // selection from candidates -> gather) needs the candidate lists and a selection small
 // enough for them; otherwise every score goes through the score workspace.
 bool use_candidates(const saga_ctx* h, int N) {
-  return h->cand_mask != nullptr && N <= kTopnCap / 4 &&
+  return h->cand_mask != nullptr && N <= kTopnSelMax && N <= kTopnCap / 4 && h->d <= kTopnMaxD &&
          (N < h->max_seq_len || h->max_seq_len <= kTopnCap);
 }
 
@@ -356,13 +360,13 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
     if ((rc = launch_bounds(h, q, k_cache, seq_lens, N))) return rc;
     if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true))) return rc;
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
-    if ((rc = launch_topn(h, q, k_cache, seq_lens, N, si, sl))) return rc;
+    if ((rc = launch_topn(h, q, k_cache, v_cache, seq_lens, N, si, sl, out))) return rc;
   } else {
     if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true))) return rc;
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     if ((rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl))) return rc;
+    if ((rc = launch_gather(h, si, sl, seq_lens, v_cache, N, out, true))) return rc;
   }
-  if ((rc = launch_gather(h, si, sl, seq_lens, v_cache, N, out, true))) return rc;
   if (prof) {
     if (record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     ++h->prof_n;

@@ -1,27 +1,35 @@
-// topn_kernel.cuh -- S2, the exact top-N of each (batch row b, query head j)
-// from the candidates that the score pass kept for it.
+// topn_kernel.cuh -- S2 to S4 of one (batch row b, query head j) from the
+// candidates that the score pass kept for it: the exact top-N, the softmax
+// over the selected logits and the gathered P.V, one CTA per row.
 //
 // Atop-N ("More Value per Key", §3.1 and App. C.1) keeps the scores at or
 // above a threshold, found by a plain compare while the scores are produced;
-// top-N itself is §2.5 Eq. (6).  The score pass (score_kernel in candidate
-// mode) kept every score >= t_lo, t_lo a lower bound for the N-th score from
-// a sample of the row's scores: per 32-position chunk c of the row a mask of
-// the passing positions, and their order-preserving keys in position order at
-// the row's slots [32c, 32c + popcount).  This kernel, one CTA per row,
-// finishes the selection exactly:
+// top-N itself is §2.5 Eq. (6), and S3/S4 are §3.1 Eq. (7).  The score pass
+// kept every score >= t_lo, t_lo a lower bound for the N-th score from a
+// sample of the row's scores: per 32-position chunk c of the row a mask of the
+// passing positions, and their order-preserving keys in position order at the
+// row's slots [32c, 32c + popcount).  This kernel:
 //   1  the chunk masks give the candidate count C and each chunk's offset (a
 //      block scan of popcounts);
 //   2  if N_b <= C <= kTopnCap the list is gathered into shared memory, in
-//      ascending position order (each thread copies the chunks of its run,
-//      eight predicated loads per chunk in flight at once);
+//      ascending position order; the first eight key slots of each chunk (one
+//      32-byte sector) are loaded in the same round as the masks, so a row
+//      costs one round of dependent loads (chunks with more than eight
+//      candidates fetch the rest afterwards);
 //   3  the N_b-th largest key T, and how many of the keys equal to T belong to
 //      the top N_b, come from an MSB-first radix select over key - min key,
 //      its first 11-bit digit aligned to the top of the keys' actual range
 //      (candidate keys share their high bits: digits of the raw key would
-//      pile them into a few bins);
+//      pile them into a few bins); once the bin holding T has at most 32
+//      keys, one warp ranks them directly;
 //   4  one ordered pass keeps every key > T and the lowest-position keys = T
-//      that are needed (block scans of tie and keep counts give each kept
-//      entry its output slot), so positions come out ascending with no sort.
+//      that are needed; one block scan of packed (greater, equal) counts gives
+//      every kept entry its output slot, so positions come out ascending with
+//      no sort; the selection goes to the caller's lists and to shared memory
+//      with its softmax weight exp(z - z_max);
+//   5  P.V: each warp gathers 32 selected value rows at a time (all loads in
+//      flight before use), fp32 accumulation, a CTA-wide sum, one division by
+//      the weight sum and one bf16 rounding.
 // The list is complete whenever C >= N_b: every score >= T is >= t_lo.  A
 // list longer than kTopnCap is selected the same way straight from the slots
 // in global memory; a list shorter than N_b (the sampled bound missed) has the
@@ -36,39 +44,47 @@
 
 namespace saga {
 
-constexpr int kTopnThreads = 512;
+constexpr int kTopnThreads = 256;
 constexpr int kTopnWarps = kTopnThreads / 32;
 constexpr int kTopnCap = 8192;                    // candidates held in shared memory
+constexpr int kTopnSelMax = 2048;                 // largest N of the candidate path
 constexpr int kTopnBins = 2048;                   // 11-bit radix digits
-constexpr int kTopnPer = 8;                       // entries per thread per step of the ordered pass
+constexpr int kTopnBinsPer = kTopnBins / kTopnThreads;   // digits owned by a thread in a scan
+constexpr int kTopnPer = 16;                      // entries per thread per step of the ordered pass
 constexpr int kTopnStep = kTopnPer * kTopnThreads;
+constexpr int kTopnRound = 4;                     // chunks per thread per round of loads
 constexpr int kTopnMaxRun = 8;                    // chunks per thread on the shared-memory path
+constexpr int kTopnMaxD = 128;
 
 // Dynamic shared memory, in 32-bit words; every region starts on a 16-byte boundary.
-constexpr int kTopnOffKey = 0;                                  // [kTopnCap] keys
-constexpr int kTopnOffPos = kTopnOffKey + kTopnCap;             // [kTopnCap] positions
-constexpr int kTopnOffHist = kTopnOffPos + kTopnCap;            // [kTopnBins]
+constexpr int kTopnOffKey = 0;                                  // [kTopnCap] candidate keys
+constexpr int kTopnOffPos = kTopnOffKey + kTopnCap;             // [kTopnCap] candidate positions
+constexpr int kTopnOffSelPos = kTopnOffPos + kTopnCap;          // [kTopnSelMax] selected positions
+constexpr int kTopnOffSelW = kTopnOffSelPos + kTopnSelMax;      // [kTopnSelMax] softmax weights
+constexpr int kTopnOffHist = kTopnOffSelW + kTopnSelMax;        // [kTopnBins]; P.V partials [warps][D]
 constexpr int kTopnOffScan = kTopnOffHist + kTopnBins;          // [kTopnWarps]
-constexpr int kTopnOffMisc = kTopnOffScan + kTopnWarps;         // [4]
-constexpr int kTopnSmemWords = kTopnOffMisc + 4;
+constexpr int kTopnOffMisc = kTopnOffScan + kTopnWarps;         // [8]
+constexpr int kTopnSmemWords = kTopnOffMisc + 8;
 constexpr size_t kTopnSmemBytes = sizeof(uint32_t) * kTopnSmemWords;
-static_assert(kTopnOffPos % 4 == 0 && kTopnOffHist % 4 == 0 && kTopnOffScan % 4 == 0 &&
-              kTopnOffMisc % 4 == 0, "shared regions on 16-byte boundaries");
+static_assert(kTopnOffPos % 4 == 0 && kTopnOffSelPos % 4 == 0 && kTopnOffSelW % 4 == 0 &&
+              kTopnOffHist % 4 == 0 && kTopnOffScan % 4 == 0 && kTopnOffMisc % 4 == 0,
+              "shared regions on 16-byte boundaries");
+static_assert(kTopnWarps * kTopnMaxD <= kTopnBins, "P.V partials fit the histogram region");
 
 struct TopnParams {
   const uint32_t* cand_mask;    // [B*h_q][mask_stride] passing positions per 32-position chunk
   long long mask_stride;
   uint32_t* zkey;               // [B*h_q][z_stride] candidate keys at their chunk slots
   long long z_stride;
-  uint32_t* gather_count;       // per-row counters of the gather kernel, reset here
   const int32_t* seq_lens;      // [B]
-  int h_q, h_k, g, L_max, N;
+  int h_q, h_k, g, h_v, g_v, L_max, N;
   int32_t* sel_idx;             // [B*h_q][N]
   float* sel_logit;             // [B*h_q][N]
-  // scoring a row again (fallback)
-  const __nv_bfloat16* q;       // [B][h_q][D]
+  const __nv_bfloat16* q;       // [B][h_q][D] (scoring a row again, fallback)
   const __nv_bfloat16* k_cache; // [B][h_k][L_max][D]
+  const __nv_bfloat16* v_cache; // [B][h_v][L_max][D]
   float scale;
+  __nv_bfloat16* out;           // [B*h_q][D]
   int* status;
 };
 
@@ -116,7 +132,7 @@ struct TopnListSrc {
 
 // The candidate slots of a row in global memory, s < n (n = 32 * chunks of
 // the row; all: every s < n = L holds the key of position s, after the row
-// was scored again).
+// was scored again by this CTA).
 struct TopnSlotSrc {
   const uint32_t* mask;
   const uint32_t* zkey;
@@ -132,13 +148,13 @@ struct TopnSlotSrc {
 };
 
 // The n_b-th largest key of the n entries of src, and in *need how many keys
-// equal to it belong to the top n_b (requires 1 <= n_b <= valid entries).
-// Radix select over d = key - kmin, MSB first, in digits of at most 11 bits,
-// the first digit ending at the top bit of kmax - kmin.  Every thread returns
-// the same values.
+// equal to it belong to the top n_b (requires 1 <= n_b <= valid entries);
+// *kmax is the largest key.  Radix select over d = key - kmin, MSB first, in
+// digits of at most 11 bits, the first digit ending at the top bit of
+// kmax - kmin.  Every thread returns the same values.
 template <class Src>
 __device__ uint32_t topn_radix(const Src& src, int n, uint32_t n_b, uint32_t* s_hist,
-                               uint32_t* s_scan, uint32_t* s_misc, uint32_t* need) {
+                               uint32_t* s_scan, uint32_t* s_misc, uint32_t* need, uint32_t* kmax_out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
   for (int i = tid; i < n; i += kTopnThreads) {
@@ -153,6 +169,7 @@ __device__ uint32_t topn_radix(const Src& src, int n, uint32_t n_b, uint32_t* s_
 #pragma unroll
   for (int w = 1; w < kTopnWarps; ++w) { kmin = min(kmin, s_hist[w]); kmax = max(kmax, s_hist[kTopnWarps + w]); }
   __syncthreads();                               // s_hist is reused below
+  *kmax_out = kmax;
   const uint32_t range = kmax - kmin;
   uint32_t prefix = 0u, pmask = 0u, k = n_b;
   int top = 32 - __clz(range);                   // bits of d still to resolve
@@ -170,75 +187,116 @@ __device__ uint32_t topn_radix(const Src& src, int n, uint32_t n_b, uint32_t* s_
       }
     }
     __syncthreads();
-    // thread t owns digits [4 (511 - t), +4): thread order runs over the digits top-down
-    const int d0 = 4 * (kTopnThreads - 1 - tid);
-    const uint32_t h0 = s_hist[d0], h1 = s_hist[d0 + 1], h2 = s_hist[d0 + 2], h3 = s_hist[d0 + 3];
-    uint32_t total;
-    uint32_t above = topn_excl_scan(h0 + h1 + h2 + h3, s_scan, total);
-    const uint32_t hs[4] = {h3, h2, h1, h0};
+    // thread t owns digits [8 (255 - t), +8): thread order runs over the digits top-down
+    const int d0 = kTopnBinsPer * (kTopnThreads - 1 - tid);
+    uint32_t h[kTopnBinsPer], c = 0u;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (above < k && above + hs[e] >= k) {     // exactly one digit of the CTA satisfies this
-        s_misc[0] = static_cast<uint32_t>(d0 + 3 - e);
+    for (int e = 0; e < kTopnBinsPer; ++e) { h[e] = s_hist[d0 + e]; c += h[e]; }
+    uint32_t total;
+    uint32_t above = topn_excl_scan(c, s_scan, total);
+#pragma unroll
+    for (int e = kTopnBinsPer - 1; e >= 0; --e) {
+      if (above < k && above + h[e] >= k) {      // exactly one digit of the CTA satisfies this
+        s_misc[0] = static_cast<uint32_t>(d0 + e);
         s_misc[1] = above;
+        s_misc[2] = h[e];
       }
-      above += hs[e];
+      above += h[e];
     }
     __syncthreads();
     const uint32_t digit = s_misc[0];
     k -= s_misc[1];
+    const uint32_t in_bin = s_misc[2];
     prefix |= digit << shift;
     pmask |= dmask << shift;
     top = shift;
     __syncthreads();                             // s_misc and s_hist are reused
+    if (top > 0 && in_bin <= 32u) {              // uniform: rank the bin's keys in one warp
+      if (tid == 0) s_misc[3] = 0u;
+      __syncthreads();
+      for (int i = tid; i < n; i += kTopnThreads) {
+        uint32_t key;
+        if (src.get(i, key) && ((key - kmin) & pmask) == prefix) s_hist[atomicAdd(&s_misc[3], 1u)] = key;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int has = lane < static_cast<int>(in_bin) ? 1 : 0;
+        const uint32_t mine = has ? s_hist[lane] : 0u;
+        uint32_t gt = 0u, ge = 0u;
+        for (int m = 0; m < static_cast<int>(in_bin); ++m) {
+          const uint32_t km = __shfl_sync(0xffffffffu, mine, m);
+          gt += km > mine ? 1u : 0u;
+          ge += km >= mine ? 1u : 0u;
+        }
+        if (has && gt < k && k <= ge) { s_misc[4] = mine; s_misc[5] = k - gt; }
+      }
+      __syncthreads();
+      const uint32_t T = s_misc[4];
+      *need = s_misc[5];
+      __syncthreads();
+      return T;
+    }
   }
   *need = k;
   return kmin + prefix;
 }
 
-// The ordered pass: entries are visited in ascending position order, eight
+// The ordered pass: entries are visited in ascending position order, kTopnPer
 // consecutive ones per thread per step; kept = key > T, or key == T among the
-// first `need` such entries.  The k-th kept entry goes to output slot k.
+// first `need` such entries, so a kept entry's slot is (keys > T before it) +
+// min(keys == T before it, need): one block scan of packed counts per step.
+// Writes the caller's lists and the shared-memory selection with its softmax
+// weight exp(z - zmax); returns this thread's sum of weights.
 template <class Src>
-__device__ void topn_emit(const Src& src, int n, uint32_t T, uint32_t need, uint32_t n_b,
-                          int32_t* idx_out, float* logit_out, uint32_t* s_scan) {
-  uint32_t ties_before = 0u, kept_before = 0u;
-  for (int base = 0; base < n && kept_before < n_b; base += kTopnStep) {   // uniform
-    const int i0 = base + kTopnPer * threadIdx.x;
+__device__ float topn_emit(const Src& src, int n, uint32_t T, uint32_t need, uint32_t n_b,
+                           float zmax, int32_t* idx_out, float* logit_out, int32_t* s_selpos,
+                           float* s_selw, uint32_t* s_scan) {
+  uint32_t gt_done = 0u, eq_done = 0u;           // counts of the earlier steps (uniform)
+  float wsum = 0.0f;
+  for (int base = 0; base < n && gt_done + min(eq_done, need) < n_b; base += kTopnStep) {
+    const int i0 = base + kTopnPer * static_cast<int>(threadIdx.x);
     uint32_t key[kTopnPer];
     bool val[kTopnPer];
-    uint32_t n_eq = 0u;
+    uint32_t ngt = 0u, neq = 0u;
 #pragma unroll
     for (int e = 0; e < kTopnPer; ++e) {
       val[e] = src.get(i0 + e, key[e]);
-      n_eq += (val[e] && key[e] == T) ? 1u : 0u;
+      ngt += (val[e] && key[e] > T) ? 1u : 0u;
+      neq += (val[e] && key[e] == T) ? 1u : 0u;
     }
-    uint32_t total_eq;
-    uint32_t r = ties_before + topn_excl_scan(n_eq, s_scan, total_eq);
-    bool keep[kTopnPer];
-    uint32_t n_keep = 0u;
+    uint32_t tot;
+    const uint32_t pre = topn_excl_scan((ngt << 16) | neq, s_scan, tot);   // step totals < 2^16
+    uint32_t gb = gt_done + (pre >> 16), qb = eq_done + (pre & 0xFFFFu);
 #pragma unroll
     for (int e = 0; e < kTopnPer; ++e) {
-      const bool tie = val[e] && key[e] == T;
-      keep[e] = val[e] && (key[e] > T || (tie && r < need));
-      r += tie ? 1u : 0u;
-      n_keep += keep[e] ? 1u : 0u;
-    }
-    uint32_t total_keep;
-    uint32_t slot = kept_before + topn_excl_scan(n_keep, s_scan, total_keep);
-#pragma unroll
-    for (int e = 0; e < kTopnPer; ++e) {
-      if (keep[e]) {
+      if (!val[e]) continue;
+      const bool gtT = key[e] > T, eqT = key[e] == T;
+      if (gtT || (eqT && qb < need)) {
+        const uint32_t slot = gb + min(qb, need);
         if (slot < n_b) {
-          idx_out[slot] = src.position(i0 + e);
-          logit_out[slot] = key_to_float(key[e]);
+          const int pos = src.position(i0 + e);
+          const float z = key_to_float(key[e]);
+          const float w = expf(z - zmax);
+          idx_out[slot] = pos;
+          logit_out[slot] = z;
+          s_selpos[slot] = pos;
+          s_selw[slot] = w;
+          wsum += w;
         }
-        ++slot;
       }
+      gb += gtT ? 1u : 0u;
+      qb += eqT ? 1u : 0u;
     }
-    ties_before += total_eq;
-    kept_before += total_keep;
+    gt_done += tot >> 16;
+    eq_done += tot & 0xFFFFu;
   }
+  return wsum;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // Keys of one row scored on CUDA cores: key(fl(fl(q . k_i) * scale)), -0 -> +0.
@@ -271,23 +329,26 @@ topn_kernel(const TopnParams p) {
   extern __shared__ __align__(16) uint32_t topn_smem[];
   uint32_t* s_key = topn_smem + kTopnOffKey;
   int32_t* s_pos = reinterpret_cast<int32_t*>(topn_smem + kTopnOffPos);
+  int32_t* s_selpos = reinterpret_cast<int32_t*>(topn_smem + kTopnOffSelPos);
+  float* s_selw = reinterpret_cast<float*>(topn_smem + kTopnOffSelW);
   uint32_t* s_hist = topn_smem + kTopnOffHist;
+  float* s_part = reinterpret_cast<float*>(topn_smem + kTopnOffHist);   // after the selection
   uint32_t* s_scan = topn_smem + kTopnOffScan;
   uint32_t* s_misc = topn_smem + kTopnOffMisc;
 
   pdl_wait();                                    // the candidate lists are complete
-  pdl_launch_dependents();                       // the gather kernel may be scheduled
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bj = blockIdx.x;
   const int b = bj / p.h_q, j = bj % p.h_q;
   const int L = p.seq_lens[b];
   const int N = p.N;
   int32_t* idx_out = p.sel_idx + static_cast<long long>(bj) * N;
   float* logit_out = p.sel_logit + static_cast<long long>(bj) * N;
-  if (tid == 0) p.gather_count[bj] = 0u;
-  if (L < 1 || L > p.L_max) {
+  __nv_bfloat16* orow = p.out + static_cast<long long>(bj) * D;
+  if (L < 1 || L > p.L_max) {                    // invalid row: padding and a zero output
     if (tid == 0) atomicOr(p.status, 0x1 /* SAGA_STATUS_BAD_SEQ_LEN */);
     for (int r = tid; r < N; r += kTopnThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
+    for (int e = tid; e < D; e += kTopnThreads) orow[e] = __float2bfloat16_rn(0.0f);
     return;
   }
   const uint32_t n_b = static_cast<uint32_t>(N < L ? N : L);
@@ -295,69 +356,155 @@ topn_kernel(const TopnParams p) {
   uint32_t* krow = p.zkey + static_cast<long long>(bj) * p.z_stride;
   const int nch = (L + 31) / 32;
 
-  // ---- candidate count and each chunk run's offset: thread t owns chunks [c0, c1)
+  // ---- candidate count and each chunk run's offset: thread t owns chunks [c0, c1);
+  // the first round also loads the first key sector of its first kTopnRound chunks
   const int cpt = (nch + kTopnThreads - 1) / kTopnThreads;
   const int c0 = min(nch, tid * cpt), c1 = min(nch, c0 + cpt);
   const bool fits = cpt <= kTopnMaxRun;
   uint32_t run_mask[kTopnMaxRun];
+  uint4 sec[kTopnRound][2];
+#pragma unroll
+  for (int u = 0; u < kTopnMaxRun; ++u) run_mask[u] = (c0 + u < c1) ? __ldcg(mrow + c0 + u) : 0u;
+#pragma unroll
+  for (int u = 0; u < kTopnRound; ++u) {
+    const uint4* kp = reinterpret_cast<const uint4*>(krow + (c0 + u) * 32);
+    sec[u][0] = (c0 + u < c1) ? __ldcg(kp) : make_uint4(0u, 0u, 0u, 0u);
+    sec[u][1] = (c0 + u < c1) ? __ldcg(kp + 1) : make_uint4(0u, 0u, 0u, 0u);
+  }
   uint32_t cnt = 0u;
 #pragma unroll
-  for (int u = 0; u < kTopnMaxRun; ++u) {
-    run_mask[u] = (u < cpt && c0 + u < c1) ? __ldcg(mrow + c0 + u) : 0u;
-    cnt += __popc(run_mask[u]);
-  }
+  for (int u = 0; u < kTopnMaxRun; ++u) cnt += __popc(run_mask[u]);
   if (!fits)
     for (int c = c0 + kTopnMaxRun; c < c1; ++c) cnt += __popc(__ldcg(mrow + c));
   uint32_t C;
   const uint32_t off = topn_excl_scan(cnt, s_scan, C);
 
-  uint32_t need;
+  uint32_t need, kmax;
+  float wsum;
   if (C >= n_b && C <= static_cast<uint32_t>(kTopnCap) && fits) {
-    // each chunk's keys are contiguous at its slots; copy them with the
-    // positions of the mask bits (up to 8 loads in flight, the rest after)
+    // Each chunk's keys are contiguous at its slots, in position order: write
+    // them with the positions of the mask bits.
     uint32_t o = off;
 #pragma unroll
-    for (int u = 0; u < kTopnMaxRun; ++u) {
-      uint32_t m = run_mask[u];
-      const int n_c = __popc(m);
-      const uint32_t* ks = krow + (c0 + u) * 32;
-      uint32_t kv[8];
+    for (int u0 = 0; u0 < kTopnMaxRun; u0 += kTopnRound) {
+      if (u0 >= cpt) break;                      // uniform
+      if (u0 > 0) {                              // rows longer than kTopnRound chunks per thread
 #pragma unroll
-      for (int e = 0; e < 8; ++e) kv[e] = (e < n_c) ? __ldcg(ks + e) : 0u;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (e < n_c) {
-          s_key[o + e] = kv[e];
-          s_pos[o + e] = (c0 + u) * 32 + (__ffs(m) - 1);
-          m &= m - 1u;
+        for (int u = 0; u < kTopnRound; ++u) {
+          const uint4* kp = reinterpret_cast<const uint4*>(krow + (c0 + u0 + u) * 32);
+          const bool live = c0 + u0 + u < c1;
+          sec[u][0] = live ? __ldcg(kp) : make_uint4(0u, 0u, 0u, 0u);
+          sec[u][1] = live ? __ldcg(kp + 1) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      for (int e = 8; e < n_c; ++e) {
-        s_key[o + e] = __ldcg(ks + e);
-        s_pos[o + e] = (c0 + u) * 32 + (__ffs(m) - 1);
-        m &= m - 1u;
+#pragma unroll
+      for (int u = 0; u < kTopnRound; ++u) {
+        uint32_t m = run_mask[u0 + u];
+        const int n_c = __popc(m);
+        const int cb = (c0 + u0 + u) * 32;
+        const uint32_t kk[8] = {sec[u][0].x, sec[u][0].y, sec[u][0].z, sec[u][0].w,
+                                sec[u][1].x, sec[u][1].y, sec[u][1].z, sec[u][1].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (e < n_c) {
+            s_key[o + e] = kk[e];
+            s_pos[o + e] = cb + (__ffs(m) - 1);
+            m &= m - 1u;
+          }
+        }
+        for (int e = 8; e < n_c; ++e) {          // rare: more than eight candidates in a chunk
+          s_key[o + e] = __ldcg(krow + cb + e);
+          s_pos[o + e] = cb + (__ffs(m) - 1);
+          m &= m - 1u;
+        }
+        o += n_c;
       }
-      o += n_c;
     }
     __syncthreads();
     const TopnListSrc src{s_key, s_pos, static_cast<int>(C)};
-    const uint32_t T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need);
-    topn_emit(src, src.n, T, need, n_b, idx_out, logit_out, s_scan);
+    const uint32_t T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need, &kmax);
+    wsum = topn_emit(src, src.n, T, need, n_b, key_to_float(kmax), idx_out, logit_out, s_selpos,
+                     s_selw, s_scan);
   } else {
     if (tid == 0) atomicOr(p.status, 0x200 /* SAGA_STATUS_INFO_ROBUST_PATH */);
     const bool all = C < n_b;                    // the bound missed: score the row again
     if (all) {
-      __syncthreads();                           // every chunk mask was read
       const __nv_bfloat16* keys =
           p.k_cache + (static_cast<long long>(b) * p.h_k + j / p.g) * p.L_max * D;
       topn_rescore<D>(p.q + static_cast<long long>(bj) * D, keys, L, p.scale, krow);
       __syncthreads();                           // the row's keys are visible to the whole CTA
     }
     const TopnSlotSrc src{mrow, krow, all ? L : nch * 32, all};
-    const uint32_t T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need);
-    topn_emit(src, src.n, T, need, n_b, idx_out, logit_out, s_scan);
+    const uint32_t T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need, &kmax);
+    wsum = topn_emit(src, src.n, T, need, n_b, key_to_float(kmax), idx_out, logit_out, s_selpos,
+                     s_selw, s_scan);
   }
   for (int r = static_cast<int>(n_b) + tid; r < N; r += kTopnThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
+
+  // ---- softmax denominator
+  wsum = warp_sum(wsum);
+  if (lane == 0) reinterpret_cast<float*>(s_scan)[warp] = wsum;
+  __syncthreads();                               // also: the selection in shared memory is complete
+  float wtot = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kTopnWarps; ++w) wtot += reinterpret_cast<const float*>(s_scan)[w];
+
+  // ---- P.V: warp w gathers slots [32 (w + 8k), +32), all 32 row loads in flight before use
+  constexpr int EPL = D / 32;                    // elements per lane: 2 or 4
+  const __nv_bfloat16* vbase = p.v_cache +
+      (static_cast<long long>(b) * p.h_v + j / p.g_v) * p.L_max * D + lane * EPL;
+  float acc[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.0f;
+  for (int g0 = warp * 32; g0 < static_cast<int>(n_b); g0 += kTopnWarps * 32) {
+    if constexpr (EPL == 4) {
+      uint2 raw[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int sl = g0 + u;
+        raw[u] = sl < static_cast<int>(n_b)
+                     ? __ldg(reinterpret_cast<const uint2*>(vbase + static_cast<long long>(s_selpos[sl]) * D))
+                     : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int sl = g0 + u;
+        const float wu = sl < static_cast<int>(n_b) ? s_selw[sl] : 0.0f;
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u].x));
+        const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u].y));
+        acc[0] = fmaf(wu, a.x, acc[0]);
+        acc[1] = fmaf(wu, a.y, acc[1]);
+        acc[2] = fmaf(wu, c.x, acc[2]);
+        acc[3] = fmaf(wu, c.y, acc[3]);
+      }
+    } else {
+      uint32_t raw[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int sl = g0 + u;
+        raw[u] = sl < static_cast<int>(n_b)
+                     ? __ldg(reinterpret_cast<const uint32_t*>(vbase + static_cast<long long>(s_selpos[sl]) * D))
+                     : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int sl = g0 + u;
+        const float wu = sl < static_cast<int>(n_b) ? s_selw[sl] : 0.0f;
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u]));
+        acc[0] = fmaf(wu, a.x, acc[0]);
+        acc[1] = fmaf(wu, a.y, acc[1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) s_part[warp * D + lane * EPL + e] = acc[e];
+  __syncthreads();
+  if (tid < D) {
+    float a = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kTopnWarps; ++w) a += s_part[w * D + tid];
+    orow[tid] = __float2bfloat16_rn(wtot > 0.0f ? a / wtot : 0.0f);
+  }
 }
 
 }  // namespace saga

@@ -272,7 +272,9 @@ def test_fused_selection_equals_stagewise():
     idx2, logit2 = dec.select(z, lens, spec.N)
     out2 = dec.combine(idx2, logit2, v, lens)
     assert torch.equal(idx, idx2) and torch.equal(logit, logit2)
-    assert torch.equal(out, out2)
+    # same selection and weights; the fused P.V sums in another order, so the
+    # two fp32 accumulations may round to neighbouring bf16 values
+    torch.testing.assert_close(out.float(), out2.float(), atol=2e-3, rtol=1e-2)
 
 
 # --------------------------------------------------------------------------- API behaviour
@@ -291,7 +293,7 @@ def test_deterministic_and_host_entry_point():
     n0 = dec.launch_count()
     dec.attn_host(q_h, k, v, l_h, spec.N, o_h)
     assert dec.status() == 0
-    assert dec.launch_count() - n0 == 5   # sample, bound, score, top-N, gather
+    assert dec.launch_count() - n0 == 4   # sample, bound, score, top-N with P.V
     assert torch.equal(o_h, a.cpu())
 
 
