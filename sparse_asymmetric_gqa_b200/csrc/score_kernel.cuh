@@ -30,8 +30,8 @@
 namespace saga {
 
 constexpr int kTileM = 128;          // positions per tile (MMA M)
-constexpr int kScoreThreads = 320;   // 10 warps: TMA, MMA, 8 x epilogue
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;        // four per TMEM lane quarter
+constexpr int kScoreThreads = 64 + 32 * kEpiWarps;   // TMA, MMA, epilogue warps
 constexpr int kMaxBatch = 1024;
 
 struct ScoreParams {
@@ -64,9 +64,11 @@ struct ScoreShape {
   static constexpr int kAccBufs = kTmemCols / kAccStride;                      // 32, 16 or 8
   // full, empty, accf[kAccBufs], acce[kAccBufs], drain
   static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
-  // Epilogue split: tile groups (alternate tiles) for up to 32 heads, else head halves.
-  static constexpr int kTileGroups = NPAD <= 32 ? 2 : 1;
-  static constexpr int kEpiHeads = NPAD * kTileGroups / 2;   // heads per epilogue warp
+  // Epilogue split of the four warps of a lane quarter: kTileGroups groups
+  // taking every kTileGroups-th tile, each group's warps splitting the heads
+  // (at most 16 per warp, 24 for a group padded to 48, so nothing spills).
+  static constexpr int kTileGroups = NPAD <= 16 ? 4 : NPAD <= 48 ? 2 : 1;
+  static constexpr int kEpiHeads = NPAD * kTileGroups / 4;   // heads per epilogue warp
   // bars, TMEM slot + abort flag, lens, unit_off
   static constexpr int kCtrlBytes = kNumBars * 8 + 16 + 2 * (kMaxBatch + 1) * 4;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kCtrlBytes;
@@ -262,13 +264,14 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
   } else {
     // ------------------------------------------------------------ epilogue
     // Warp w reads TMEM lane quarter w % 4 (the hardware rule); its set
-    // (w - 2) / 4 takes the items of that parity (two tile groups) or the
-    // heads [set * H, set * H + H) of every item (one tile group).
+    // (w - 2) / 4 gives its tile group (set % TG: the tiles i with i % TG equal
+    // to it) and its heads [h0, h0 + H), h0 = (set / TG) * H.
     constexpr int H = S::kEpiHeads;
     constexpr int TG = S::kTileGroups;
     const int quad = warp & 3;
     const int set = (warp - 2) >> 2;
-    const int h0 = (TG == 1) ? set * H : 0;
+    const int tg = set % TG;
+    const int h0 = (set / TG) * H;
     const uint64_t pol_z = policy_evict_last();
     bool alive = true;
     // Item i's accumulator, heads h0 .. h0 + H - 1 of this lane's position.
@@ -324,7 +327,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
       c.seek(u0, unit_off, lens, p.B, p.h_k);
       for (int jt = 0; jt < n_tiles; ++jt, c.next(unit_off, lens, p.B, p.h_k)) {
         const int i = jt;                         // index in the pipeline
-        if (!alive || (TG == 2 && (i & 1) != set)) continue;
+        if (!alive || i % TG != tg) continue;
         if (c.b != seg_b || c.kh != seg_kh) {     // a new row segment
           if (!kCand) flush();
           seg_b = c.b;
