@@ -28,6 +28,8 @@
  *   scores    fp32  [B][h_q][stride] z for positions < L_b (stride >= L_max)
  * B is the handle's current batch (saga_decode_set_batch; initially max_batch);
  * L_max is the handle's max_seq_len, which is also the caches' position stride.
+ * q, k_cache and v_cache start on 16-byte boundaries (any cudaMalloc'd buffer
+ * does); a base that does not is rejected with SAGA_ERR_INVALID_ARG.
  *
  * Ownership: every tensor argument is caller-owned; the library never frees or
  * retains it past the call.  The handle owns only its workspace (score rows,
@@ -67,7 +69,8 @@ extern "C" {
 
 /* Return codes. */
 #define SAGA_OK               0
-#define SAGA_ERR_INVALID_ARG  1  /* null pointer, bad size, mismatched heads, N > max_N ... */
+#define SAGA_ERR_INVALID_ARG  1  /* null pointer, bad size, mismatched heads, N > max_N, a q /
+                                     k_cache / v_cache base not 16-byte aligned ... */
 #define SAGA_ERR_UNSUPPORTED  2  /* valid but not built: d not in {64,128}, g > 64, wrong GPU */
 #define SAGA_ERR_CUDA         3  /* a CUDA runtime/driver call failed */
 #define SAGA_ERR_DEVICE       4  /* saga_decode_status found an error bit set */

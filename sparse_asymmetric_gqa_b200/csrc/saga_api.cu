@@ -334,6 +334,10 @@ struct DeviceGuard {   // run a call on the handle's device, restore the caller'
   }
 };
 
+// q, the caches and the score rows are read with 16-byte vector loads, TMA and
+// asynchronous copies: their base addresses must be 16-byte aligned.
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 // The candidate path (sampled bounds -> score pass with fused compare ->
 // selection from candidates -> gather) needs the candidate lists and a selection small
 // enough for them; otherwise every score goes through the score workspace.
@@ -345,6 +349,7 @@ bool use_candidates(const saga_ctx* h, int N) {
 int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
                 const int32_t* seq_lens, int N, void* out, int32_t* sel_idx, float* sel_logit) {
   if (!q || !k_cache || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
@@ -504,6 +509,7 @@ int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache
   if (!h) return SAGA_ERR_INVALID_ARG;
   if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
   if (!q_host || !seq_lens_host || !out_host || !k_cache || !v_cache) return SAGA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
@@ -524,6 +530,7 @@ int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache
 int saga_score(saga_handle h, const void* q, const void* k_cache, const int32_t* seq_lens,
                int h_q, int h_k, int head_dim, float* scores, int scores_stride) {
   if (!h || !q || !k_cache || !seq_lens || !scores) return SAGA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache)) return SAGA_ERR_INVALID_ARG;
   if (h_q != h->h_q || h_k != h->h_k || head_dim != h->d) return SAGA_ERR_INVALID_ARG;
   if (scores_stride < h->max_seq_len) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
@@ -545,6 +552,7 @@ int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
                  const void* v_cache, const int32_t* seq_lens, int h_q, int h_v, int head_dim,
                  int N, void* out) {
   if (!h || !sel_idx || !sel_logit || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (!aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
   if (h_q != h->h_q || h_v != h->h_v || head_dim != h->d) return SAGA_ERR_INVALID_ARG;
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
@@ -680,6 +688,7 @@ int saga_combine_noalloc(const int32_t* sel_idx, const float* sel_logit, const v
                          const int32_t* seq_lens, int batch, int max_seq_len, int h_q, int h_v,
                          int head_dim, int N, void* out, void* cuda_stream) {
   if (!sel_idx || !sel_logit || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (!aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
   if (batch < 1 || max_seq_len < 1 || h_q < 1 || h_v < 1 || N < 1) return SAGA_ERR_INVALID_ARG;
   if (h_q % h_v != 0) return SAGA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return SAGA_ERR_UNSUPPORTED;

@@ -71,6 +71,14 @@ def test_null_handle_rejected(lib):
     assert lib.saga_decode_status(None, ctypes.byref(v)) == _lib.SAGA_ERR_INVALID_ARG
 
 
+def test_unaligned_value_cache_rejected_before_cuda(lib):
+    # v_cache must start on a 16-byte boundary; the check comes before any CUDA call
+    fake = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    rc = lib.saga_combine_noalloc(fake, fake, odd, fake, 1, 64, 8, 2, 128, 16, fake, None)
+    assert rc == _lib.SAGA_ERR_INVALID_ARG
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
