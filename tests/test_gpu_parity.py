@@ -170,6 +170,28 @@ def test_all_equal_scores_take_lowest_positions():
             assert_out_close(to_np(out[b, j]), mean_v, f"row ({b},{j})")
 
 
+def test_bound_that_misses_rescores_the_row():
+    # Adversarial for the sampled bound: query-aligned keys exactly at the 1024
+    # sampled positions (32 blocks of 32 at 32 * floor(blk * (L / 32) / 32)),
+    # small keys elsewhere, and N = 2048.  The bound lands among the planted
+    # scores, fewer than N_b scores pass it, and the row must be scored again
+    # and selected exactly (INFO_ROBUST_PATH).
+    B, L, h_q, h_k, h_v, d, N = 1, 16384, 4, 1, 2, 64, 2048
+    inp = make_raw(11, B, L, [L], h_q, h_k, h_v, d)
+    inp.q[:] = inp.q[:, :1]                               # one query for all four heads
+    inp.k_cache.mul_(0.1)
+    lpb = L // 32
+    sampled = [32 * ((blk * lpb) // 32) + i for blk in range(32) for i in range(32)]
+    inp.k_cache[0, 0, sampled] = (3.0 * inp.q[0, 0].float()).to(torch.bfloat16)
+    dec = SagaDecoder(B, L, h_q, h_k, h_v, d, N)
+    out, idx, logit, st = run_decode(dec, *_dev(inp), N)
+    assert st & _lib.SAGA_STATUS_INFO_ROBUST_PATH
+    assert st & 0xFF == 0
+    sel = set(idx[0, 0].tolist())
+    assert set(sampled) <= sel                            # every planted key is selected
+    check_rows(inp, h_q, h_k, h_v, N, out, idx, logit, [(0, j) for j in range(h_q)])
+
+
 def test_bad_seq_lens_flagged_and_zeroed():
     B, L, h_q, h_k, h_v, d, N = 3, 1024, 4, 1, 2, 64, 64
     inp = make_raw(9, B, L, [0, 700, L + 5], h_q, h_k, h_v, d)
