@@ -30,7 +30,7 @@
 namespace saga {
 
 constexpr int kTileM = 128;          // positions per tile (MMA M)
-constexpr int kEpiWarps = 16;        // four per TMEM lane quarter
+constexpr int kEpiWarps = 8;         // two per TMEM lane quarter
 constexpr int kScoreThreads = 64 + 32 * kEpiWarps;   // TMA, MMA, epilogue warps
 constexpr int kMaxBatch = 1024;
 
@@ -64,11 +64,11 @@ struct ScoreShape {
   static constexpr int kAccBufs = kTmemCols / kAccStride;                      // 32, 16 or 8
   // full, empty, accf[kAccBufs], acce[kAccBufs], drain
   static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
-  // Epilogue split of the four warps of a lane quarter: kTileGroups groups
-  // taking every kTileGroups-th tile, each group's warps splitting the heads
-  // (at most 16 per warp, 24 for a group padded to 48, so nothing spills).
-  static constexpr int kTileGroups = NPAD <= 16 ? 4 : NPAD <= 48 ? 2 : 1;
-  static constexpr int kEpiHeads = NPAD * kTileGroups / 4;   // heads per epilogue warp
+  // Epilogue split of the kEpiWarps / 4 warps of a lane quarter: kTileGroups
+  // groups taking every kTileGroups-th tile, each group's warps splitting the
+  // heads (two tile groups for up to 32 heads, else head halves).
+  static constexpr int kTileGroups = NPAD <= 32 ? 2 : 1;
+  static constexpr int kEpiHeads = NPAD * kTileGroups / (kEpiWarps / 4);   // heads per warp
   // bars, TMEM slot + abort flag, lens, unit_off
   static constexpr int kCtrlBytes = kNumBars * 8 + 16 + 2 * (kMaxBatch + 1) * 4;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kCtrlBytes;
