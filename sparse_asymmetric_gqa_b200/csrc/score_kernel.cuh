@@ -107,6 +107,9 @@ struct TileCursor {
 __device__ __forceinline__ void st_global_hint(float* p, float v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" :: "l"(p), "f"(v), "l"(pol) : "memory");
 }
+__device__ __forceinline__ void st_global_hint(uint32_t* p, uint32_t v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" :: "l"(p), "r"(v), "l"(pol) : "memory");
+}
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
   *abort_flag = 1;
@@ -355,10 +358,12 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const bool take = valid && h0 + e < p.g && zz >= tl[e];
             const uint32_t m = __ballot_sync(0xffffffffu, take);
             if (lane == e) my_m = m;
-            if (take) kslot[e * p.z_stride + __popc(m & lt)] = ordered_key(zz);
+            // candidates are written L2-evict-last (the K stream is evict-first), so
+            // that the selector finds them in L2
+            if (take) st_global_hint(kslot + e * p.z_stride + __popc(m & lt), ordered_key(zz), pol_z);
           }
           if (lane < H && h0 + lane < p.g && chunk * 32 < c.Lb)   // lane e: head e's mask
-            p.cand_mask[static_cast<long long>(row0 + lane) * p.mask_stride + chunk] = my_m;
+            st_global_hint(p.cand_mask + static_cast<long long>(row0 + lane) * p.mask_stride + chunk, my_m, pol_z);
         } else if (valid) {
           float* zrow = p.z + static_cast<long long>(row0) * p.z_stride + pos;
 #pragma unroll
