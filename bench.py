@@ -405,9 +405,9 @@ def run_saga(args, rank, world, local):
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
-            "kernel": "score pass: sample_kernel + bound_kernel + score_kernel (S1, q.K over the "
-                      "whole key cache, with the candidate compare; the score kernel streams K "
-                      "while the two small bound kernels run)",
+            "kernel": "score_kernel (S1, q.K over the whole key cache with the candidate "
+                      "compare; bracketed by events in a separate profiled graph, where it does "
+                      "not start early under the bound kernels)",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": traffic,
             "algorithmic_bytes_per_launch": k_bytes, "avg_launch_us": score_avg_s * 1e6,

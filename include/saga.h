@@ -190,8 +190,10 @@ SAGA_API int saga_decode_status(saga_handle h, int* device_status);
 SAGA_API int saga_decode_launch_count(saga_handle h, long long* count);
 
 /* Profiling: when enabled, each decode call records CUDA events around its
- * score pass (threshold + score kernels) and around the whole call on the
- * handle's stream (up to max_calls calls; inside CUDA-graph capture the
+ * score kernel and around the whole call on the handle's stream (the record
+ * before the score kernel keeps it from starting early under programmatic
+ * dependent launch, so the interval is the kernel's own duration; up to
+ * max_calls calls; inside CUDA-graph capture the
  * records become graph nodes, so every replay re-records them; the events
  * live until the handle is freed).  Disabling stops recording and keeps the
  * events.  saga_decode_profile_read synchronises and returns the summed

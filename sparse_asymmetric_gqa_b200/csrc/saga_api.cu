@@ -98,7 +98,7 @@ struct saga_ctx {
   // profiling
   bool prof = false;
   int prof_max = 0, prof_n = 0;
-  std::vector<cudaEvent_t> ev;   // 3 per recorded call: start, after score, end
+  std::vector<cudaEvent_t> ev;   // 4 per recorded call: start, score start, score end, end
 };
 
 namespace {
@@ -354,7 +354,7 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
   const bool prof = h->prof && h->prof_n < h->prof_max;
-  cudaEvent_t* ev = prof ? &h->ev[3 * h->prof_n] : nullptr;
+  cudaEvent_t* ev = prof ? &h->ev[4 * h->prof_n] : nullptr;
   // The selection goes to the caller's arrays when given, else to the workspace
   // (row stride N either way).
   int32_t* si = sel_idx ? sel_idx : h->sel_idx;
@@ -363,17 +363,19 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   int rc;
   if (use_candidates(h, N)) {
     if ((rc = launch_bounds(h, q, k_cache, seq_lens, N))) return rc;
-    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true))) return rc;
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true))) return rc;
+    if (prof && record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     if ((rc = launch_topn(h, q, k_cache, v_cache, seq_lens, N, si, sl, out))) return rc;
   } else {
-    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true))) return rc;
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true))) return rc;
+    if (prof && record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     if ((rc = launch_select(h, h->z, h->z_stride, true, seq_lens, N, si, sl))) return rc;
     if ((rc = launch_gather(h, si, sl, seq_lens, v_cache, N, out, true))) return rc;
   }
   if (prof) {
-    if (record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (record_event(ev[3], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     ++h->prof_n;
   }
   return SAGA_OK;
@@ -593,10 +595,10 @@ int saga_decode_profile(saga_handle h, int enable, int max_calls) {
     h->prof = false;
     return SAGA_OK;
   }
-  if (h->ev.size() < 3 * static_cast<size_t>(max_calls)) {
+  if (h->ev.size() < 4 * static_cast<size_t>(max_calls)) {
     if (cudaStreamSynchronize(h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
-    h->ev.assign(3 * static_cast<size_t>(max_calls), nullptr);
+    h->ev.assign(4 * static_cast<size_t>(max_calls), nullptr);
     for (auto& e : h->ev)
       if (cudaEventCreate(&e) != cudaSuccess) return SAGA_ERR_CUDA;
   }
@@ -614,8 +616,8 @@ int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms, i
   double s = 0.0, c = 0.0;
   for (int i = 0; i < h->prof_n; ++i) {
     float a = 0.0f, b = 0.0f;
-    if (cudaEventElapsedTime(&a, h->ev[3 * i], h->ev[3 * i + 1]) != cudaSuccess) return SAGA_ERR_CUDA;
-    if (cudaEventElapsedTime(&b, h->ev[3 * i], h->ev[3 * i + 2]) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (cudaEventElapsedTime(&a, h->ev[4 * i + 1], h->ev[4 * i + 2]) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (cudaEventElapsedTime(&b, h->ev[4 * i], h->ev[4 * i + 3]) != cudaSuccess) return SAGA_ERR_CUDA;
     s += a;
     c += b;
   }

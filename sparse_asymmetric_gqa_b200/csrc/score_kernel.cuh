@@ -57,8 +57,11 @@ struct ScoreShape {
   static constexpr int kAPart = kTileM * 128;           // 16 KB of K per atom
   static constexpr int kBPart = NPAD * 128;             // q rows per atom
   static constexpr int kStageBytes = kParts * (kAPart + kBPart);
+  // 128 KB of K in flight per SM (four stages for d = 128) measured faster than
+  // 160 or 192 KB: more bytes in flight only lengthened the memory queues.
   static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
-  static constexpr int kStages = kStagesRaw < 8 ? kStagesRaw : 8;
+  static constexpr int kStagesK = (128 * 1024) / (kParts * kAPart);
+  static constexpr int kStages = kStagesRaw < kStagesK ? kStagesRaw : kStagesK;
   static constexpr int kAccStride = NPAD <= 16 ? 16 : NPAD <= 32 ? 32 : 64;   // columns per accumulator
   static constexpr int kTmemCols = 512;                                        // all of TMEM
   static constexpr int kAccBufs = kTmemCols / kAccStride;                      // 32, 16 or 8
