@@ -5,6 +5,10 @@ import this package; the CUDA path never does.
 """
 from .saga_oracle import (head_maps, scores, top_n, nth_score, softmax_selected,
                           gathered_pv, decode_row, decode_attn, combine)
+from .atopn_oracle import (calibrate_tau, tail_max, step_threshold, step_select,
+                           step_row, calibrate_row, step_attn)
 
 __all__ = ["head_maps", "scores", "top_n", "nth_score", "softmax_selected",
-           "gathered_pv", "decode_row", "decode_attn", "combine"]
+           "gathered_pv", "decode_row", "decode_attn", "combine",
+           "calibrate_tau", "tail_max", "step_threshold", "step_select",
+           "step_row", "calibrate_row", "step_attn"]
