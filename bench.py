@@ -280,6 +280,18 @@ def run_saga(args, rank, world, local):
     status = dec.status()
     if status & 0xFF:
         raise RuntimeError(f"device status 0x{status:x}")
+    # value rows one call really reads: the union over the query heads that share a value head
+    x0 = layers[0]
+    sel = torch.empty(B, spec.h_q, spec.N, dtype=torch.int32, device=dev)
+    dec.attn(x0.q, x0.k_cache, x0.v_cache, x0.seq_lens, spec.N, out=outs[0], sel_idx=sel,
+             sel_logit=torch.empty(B, spec.h_q, spec.N, dtype=torch.float32, device=dev))
+    g_v = spec.h_q // spec.h_v
+    unique_rows = 0
+    for b in range(B):
+        for vh in range(spec.h_v):
+            ids = sel[b, vh * g_v:(vh + 1) * g_v].flatten()
+            unique_rows += int(torch.unique(ids[ids >= 0]).numel())
+    v_bytes_unique = unique_rows * spec.head_dim * 2
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(side):
@@ -419,6 +431,7 @@ def run_saga(args, rank, world, local):
             "model": "K cache over valid positions + N V rows per value head",
             "profiled_graph_ms_per_step": prof_ms / args.steps,
             "v_bytes_per_query_head_model": v_bytes_per_head,
+            "v_bytes_unique_rows_measured": v_bytes_unique,
         },
         "cpu_baseline": {
             "value": cpu_tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",

@@ -95,7 +95,7 @@ typedef struct saga_ctx* saga_handle;
  * head_dim, and selections of up to max_N positions.  cuda_stream is a
  * cudaStream_t (NULL = legacy default stream).  The current CUDA device at
  * this call is the handle's device.  Workspace: about
- * 4*max_batch*h_q*(round_up(max_seq_len,32) + 2*max_N + 3 +
+ * 4*max_batch*h_q*(round_up(max_seq_len,32)*17/16 + 4*max_N + 1030 +
  * ceil(min(max_N,max_seq_len)/256)*(head_dim+2)) bytes.
  * Returns SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_CUDA. */
 SAGA_API int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len,
@@ -122,6 +122,41 @@ SAGA_API int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cac
                         const void* v_cache, const int32_t* seq_lens,
                         int h_q, int h_k, int h_v, int head_dim, int N, void* out,
                         int32_t* sel_idx, float* sel_logit);
+
+/* Stateful Atop-N ([MVK] §3.1, App. C.1): a per-row probability threshold tau,
+ * calibrated on one decode step and reused by the following ones (the paper
+ * recalibrates every n = 32 steps; when is the caller's choice).  The state is
+ * the caller's device array log_tau, fp32 [B][h_q], natural log of tau.
+ *
+ * saga_atopn_calibrate: the decode step of saga_decode_attn_ex (exact top-N,
+ * out, optional sel_idx / sel_logit [B][h_q][N]), and for every row
+ * log_tau[b][j] = z_(N_b) - log(sum_i exp(z_i)): the log of the softmax
+ * probability of the N_b-th largest score (N_b = min(N, L_b)).  A row with an
+ * invalid seq_len gets log_tau = -inf.
+ *
+ * saga_atopn_step: with t = log_tau[b][j] + log(sum_i exp(z_i)) (the paper's
+ * m_hat + log(tau * s_hat), in which the reference m_hat cancels), selects every
+ * position with z_i >= t in ascending position order, keeps the first 2N (the
+ * paper drops the excess in arbitrary order; the lowest positions are kept
+ * here, so results are reproducible), and computes the softmax over the kept
+ * logits and the gathered P.V into out.  sel_idx / sel_logit, if given, are
+ * [B][h_q][2N], padded with -1 / -inf.  A row where nothing reaches t gets a
+ * zero output; a NaN log_tau counts as -inf (every position passes).
+ *
+ * Both: same layouts, ownership and errors as saga_decode_attn_ex; log_tau
+ * non-NULL device pointer; 1 <= N <= min(max_N, 2048), else
+ * SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED.  The log-sum-exp runs over all
+ * L_b scores in fp32; a row whose scores leave the fp32 range of its sums, or
+ * whose sampled candidate bound lies above t, is scored again on CUDA cores
+ * (SAGA_STATUS_INFO_ROBUST_PATH). */
+SAGA_API int saga_atopn_calibrate(saga_handle h, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* seq_lens, int h_q, int h_k,
+                                  int h_v, int head_dim, int N, void* out, int32_t* sel_idx,
+                                  float* sel_logit, float* log_tau);
+SAGA_API int saga_atopn_step(saga_handle h, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* seq_lens, int h_q, int h_k,
+                             int h_v, int head_dim, int N, const float* log_tau, void* out,
+                             int32_t* sel_idx, float* sel_logit);
 
 /* The decode step with the per-step inputs and result in HOST memory:
  * q_host (bf16 [B][h_q][d]) and seq_lens_host (int32 [B]) are copied to the

@@ -28,7 +28,11 @@ Readings where the pages leave the step open (also in the design notes):
 * the collected positions are listed in ascending order; unused slots are
   padding (index -1, logit -inf);
 * calibration with N >= L_b gives tau = the smallest probability (every
-  position passes).
+  position passes);
+* a step where no entry reaches the threshold (tau above the row's largest
+  probability) selects nothing and gives a zero output (a softmax over an
+  all-padding buffer has no value; the zero row is the convention of the
+  library's combine stage for a row with no valid entry).
 
 Parity pins (``tests/test_atopn_oracle.py``): a step with tau calibrated on the
 same scores selects exactly the top-N for any tail (t reduces to the N-th
@@ -77,6 +81,8 @@ def step_row(q_j, keys, values, tau: float, tail: int, cap: int):
     z = keys.astype(np.float64) @ q_j.astype(np.float64) / np.sqrt(d)
     idx = step_select(z, tau, tail, cap)
     z_sel = z[idx]
+    if idx.size == 0:
+        return np.zeros(values.shape[1]), idx, z_sel
     p = np.exp(z_sel - z_sel.max())
     p /= p.sum()
     out = p @ values[idx].astype(np.float64)

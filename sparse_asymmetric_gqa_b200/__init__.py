@@ -106,6 +106,55 @@ class SagaDecoder:
                        self.lib.saga_decode_attn_ex(*args, _ptr(sel_idx), _ptr(sel_logit)))
         return out
 
+    def atopn_calibrate(self, q, k_cache, v_cache, seq_lens, N: int, log_tau=None, out=None,
+                        sel_idx=None, sel_logit=None):
+        """Calibration step of stateful Atop-N: the exact top-N decode step, and per row
+        log tau = log of the softmax probability of the N-th largest score.
+
+        Returns (out, log_tau); log_tau is fp32 [B, h_q], the state that later
+        ``atopn_step`` calls reuse.
+        """
+        self._check_caches(q, k_cache, v_cache, seq_lens)
+        B = self.batch
+        if out is None:
+            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
+        if log_tau is None:
+            log_tau = torch.empty(B, self.h_q, dtype=torch.float32, device=q.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+        _need(log_tau, "log_tau", torch.float32, (B, self.h_q), "cuda")
+        if sel_idx is not None:
+            _need(sel_idx, "sel_idx", torch.int32, (B, self.h_q, N), "cuda")
+        if sel_logit is not None:
+            _need(sel_logit, "sel_logit", torch.float32, (B, self.h_q, N), "cuda")
+        self._stream()
+        _lib.check("saga_atopn_calibrate", self.lib.saga_atopn_calibrate(
+            self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), self.h_q, self.h_k,
+            self.h_v, self.head_dim, N, _ptr(out), _ptr(sel_idx), _ptr(sel_logit), _ptr(log_tau)))
+        return out, log_tau
+
+    def atopn_step(self, q, k_cache, v_cache, seq_lens, N: int, log_tau, out=None,
+                   sel_idx=None, sel_logit=None):
+        """A step of stateful Atop-N: keep every score z >= log_tau + logsumexp(z) (the
+        first 2N positions), softmax over them and the gathered P.V.
+
+        sel_idx / sel_logit, if given, are [B, h_q, 2N] (padding -1 / -inf).
+        """
+        self._check_caches(q, k_cache, v_cache, seq_lens)
+        B = self.batch
+        if out is None:
+            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+        _need(log_tau, "log_tau", torch.float32, (B, self.h_q), "cuda")
+        if sel_idx is not None:
+            _need(sel_idx, "sel_idx", torch.int32, (B, self.h_q, 2 * N), "cuda")
+        if sel_logit is not None:
+            _need(sel_logit, "sel_logit", torch.float32, (B, self.h_q, 2 * N), "cuda")
+        self._stream()
+        _lib.check("saga_atopn_step", self.lib.saga_atopn_step(
+            self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), self.h_q, self.h_k,
+            self.h_v, self.head_dim, N, _ptr(log_tau), _ptr(out), _ptr(sel_idx), _ptr(sel_logit)))
+        return out
+
     def attn_host(self, q_host, k_cache, v_cache, seq_lens_host, N: int, out_host):
         """Decode step with q / seq_lens / out in (pinned) host memory; asynchronous."""
         B = self.batch

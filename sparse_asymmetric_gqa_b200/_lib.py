@@ -28,6 +28,8 @@ SIGNATURES = {
     "saga_decode_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "saga_decode_attn_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "saga_decode_attn_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "saga_atopn_calibrate": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "saga_atopn_step": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "saga_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I]),
     "saga_select": (_I, [_P, _P, _I, _P, _I, _I, _P, _P]),
     "saga_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),

@@ -23,6 +23,12 @@
 // The number of samples above the true N_b-th score has mean r_s, so the bound
 // lies below it unless that count exceeds its mean by about six standard
 // deviations.  Rows that the selector takes whole get t_lo = -inf.
+//
+// The bound kernel also writes m_ref, the largest sampled score of the row
+// (+inf for rows without a sample): the reference that the score pass
+// subtracts before it sums exp(z) over the row for the log-sum-exp of the
+// calibrated threshold (App. C.1 takes the largest score of a tail of the row;
+// the reference cancels from the threshold, it only keeps the sum in range).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -44,6 +50,7 @@ struct BoundParams {
   float scale;
   float* samp;                   // [B*h_q][kSampleSize] scratch
   float* t_lo;                   // [B*h_q]
+  float* m_ref;                  // [B*h_q] largest sampled score, or nullptr
 };
 
 // Rows whose candidates are every position (t_lo = -inf), or invalid rows.
@@ -123,8 +130,25 @@ bound_kernel(const BoundParams p) {
   const int bj = blockIdx.x;
   const int L = p.seq_lens[bj / p.h_q];
   if (bound_takes_all(L, p)) {
-    if (lane == 0) p.t_lo[bj] = -INFINITY;
+    if (lane == 0) {
+      p.t_lo[bj] = -INFINITY;
+      if (p.m_ref) p.m_ref[bj] = INFINITY;
+    }
     return;
+  }
+  const float* srow = p.samp + static_cast<long long>(bj) * kSampleSize;
+  constexpr int kPer = kSampleSize / 32;
+  uint32_t key[kPer];
+  uint32_t kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    key[i] = ordered_key(__fadd_rn(__ldcg(srow + i * 32 + lane), 0.0f));
+    kmax = max(kmax, key[i]);
+    key[i] >>= 16;
+  }
+  if (p.m_ref) {
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) p.m_ref[bj] = key_to_float(kmax);
   }
   const int n_b = p.N < L ? p.N : L;
   const float rs = static_cast<float>(n_b) * kSampleSize / static_cast<float>(L);
@@ -134,11 +158,6 @@ bound_kernel(const BoundParams p) {
     return;
   }
   const uint32_t r = static_cast<uint32_t>(rf);
-  const float* srow = p.samp + static_cast<long long>(bj) * kSampleSize;
-  constexpr int kPer = kSampleSize / 32;
-  uint32_t key[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) key[i] = ordered_key(__fadd_rn(__ldcg(srow + i * 32 + lane), 0.0f)) >> 16;
   uint32_t T = 0u;                                // the largest 16-bit key with >= r samples at or above it
   for (int bit = 15; bit >= 0; --bit) {
     const uint32_t trial = T | (1u << bit);

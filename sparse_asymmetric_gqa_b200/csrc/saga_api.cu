@@ -1,11 +1,19 @@
 // saga_api.cu -- the C ABI declared in include/saga.h: argument validation,
 // the handle and its workspace, TMA descriptor encoding and the launch plan.
 //
-// One decode call enqueues three kernels on the handle's stream:
-//   score_kernel   S1, persistent, one CTA per SM (tcgen05 + TMA)
+// A decode call enqueues four kernels on the handle's stream (the candidate path):
+//   sample_kernel  1024 sampled scores per (batch row, query head), CUDA cores
+//   bound_kernel   a lower bound t_lo for the selection threshold of each row
+//   score_kernel   S1, persistent, one CTA per SM (tcgen05 + TMA), keeping the
+//                  scores >= t_lo as candidates
+//   topn_kernel    S2 + S3 + S4 from the candidates, one CTA per (b, j)
+// The calibration call and a step of stateful Atop-N run the same four, the
+// score pass also summing exp(z - m_ref) per chunk for the row's log-sum-exp.
+// Selections wider than the candidate path takes (N > 2048) run three:
+//   score_kernel   S1, every score to the workspace
 //   select_kernel  S2, one CTA per (batch row, query head)
 //   gather_kernel  S3 + S4, one CTA per 256 selected rows of a (b, j)
-// Nothing is allocated, synchronised or copied to the host on that path.
+// Nothing is allocated, synchronised or copied to the host on either path.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -91,6 +99,8 @@ struct saga_ctx {
   long long mask_stride = 0;      // z_stride / 32
   float* samp = nullptr;          // sampled scores [rows][kSampleSize]
   float* t_lo = nullptr;          // candidate bounds [rows]
+  float* m_ref = nullptr;         // exp-sum references [rows] (calibration and steps)
+  float* lse_part = nullptr;      // chunk sums of exp(z - m_ref) [rows][mask_stride]
   float* partial = nullptr;       // gather partials [rows][max_chunks][d + 2]
   uint32_t* counter = nullptr;    // gather merge counters [rows]
   int max_chunks = 0;
@@ -114,6 +124,9 @@ int set_smem_attrs_once() {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes); \
   if (e == cudaSuccess)                                                                           \
     e = cudaFuncSetAttribute(score_kernel<D, NP, true>,                                           \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes); \
+  if (e == cudaSuccess)                                                                           \
+    e = cudaFuncSetAttribute(score_kernel<D, NP, true, true>,                                     \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes);
     SAGA_ATTR(64, 16) SAGA_ATTR(64, 32) SAGA_ATTR(64, 48) SAGA_ATTR(64, 64)
     SAGA_ATTR(128, 16) SAGA_ATTR(128, 32) SAGA_ATTR(128, 48) SAGA_ATTR(128, 64)
@@ -121,12 +134,15 @@ int set_smem_attrs_once() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sizeof(SelectSmem)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kTopnSmemBytes));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kTopnSmemBytes));
+#define SAGA_TOPN_ATTR(D, M, S)                                                                   \
+  if (e == cudaSuccess)                                                                           \
+    e = cudaFuncSetAttribute(topn_kernel<D, M, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                             static_cast<int>(TopnLayout<S>::kBytes));
+    SAGA_TOPN_ATTR(64, kModeExact, kTopnSelNarrow) SAGA_TOPN_ATTR(128, kModeExact, kTopnSelNarrow)
+    SAGA_TOPN_ATTR(64, kModeCalibrate, kTopnSelNarrow) SAGA_TOPN_ATTR(128, kModeCalibrate, kTopnSelNarrow)
+    SAGA_TOPN_ATTR(64, kModeStep, kTopnSelNarrow) SAGA_TOPN_ATTR(128, kModeStep, kTopnSelNarrow)
+    SAGA_TOPN_ATTR(64, kModeStep, kTopnSelMax) SAGA_TOPN_ATTR(128, kModeStep, kTopnSelMax)
+#undef SAGA_TOPN_ATTR
     rc = (e == cudaSuccess) ? 0 : 1;
   });
   return rc;
@@ -165,7 +181,7 @@ cudaError_t launch(saga_ctx* h, void (*kernel)(KArgs...), dim3 grid, dim3 block,
 // candidate keys in the workspace; a programmatic dependent of the bound
 // kernel); otherwise every score goes to z.
 int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
-                 float* z, long long z_stride, bool stats, bool cand = false) {
+                 float* z, long long z_stride, bool stats, bool cand = false, bool lse = false) {
   CUtensorMap mk, mq;
   const uint64_t k_rows = static_cast<uint64_t>(h->batch) * h->h_k * h->max_seq_len;
   const uint64_t q_rows = static_cast<uint64_t>(h->batch) * h->h_q;
@@ -178,6 +194,8 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
   p.cand_mask = h->cand_mask;
   p.mask_stride = h->mask_stride;
   p.t_lo = h->t_lo;
+  p.m_ref = h->m_ref;
+  p.lse_part = (cand && lse) ? h->lse_part : nullptr;
   p.stat_min = (stats && !cand) ? h->stat_min : nullptr;
   p.stat_max = (stats && !cand) ? h->stat_max : nullptr;
   p.status = h->status;
@@ -194,7 +212,9 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
   cudaError_t e = cudaErrorInvalidValue;
 #define SAGA_CASE(D, NP)                                                                       \
   if (h->d == D && h->npad == NP)                                                              \
-    e = cand ? launch(h, score_kernel<D, NP, true>, dim3(grid), dim3(kScoreThreads),           \
+    e = (cand && lse) ? launch(h, score_kernel<D, NP, true, true>, dim3(grid), dim3(kScoreThreads), \
+                               ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p)                  \
+      : cand ? launch(h, score_kernel<D, NP, true>, dim3(grid), dim3(kScoreThreads),           \
                       ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p)                          \
              : launch(h, score_kernel<D, NP, false>, dim3(grid), dim3(kScoreThreads),          \
                       ScoreShape<D, NP>::kSmemBytes, kPlain, mk, mq, p);
@@ -204,9 +224,11 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
-// Candidate bounds: the sample kernel (after the previous kernel in the stream)
-// and the bound kernel (a programmatic dependent of it).
-int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens, int N) {
+// Candidate bounds for the n_target largest scores of each row: the sample
+// kernel (after the previous kernel in the stream) and the bound kernel (a
+// programmatic dependent of it); with ref, also the exp-sum references.
+int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
+                  int n_target, bool ref) {
   BoundParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
@@ -215,11 +237,12 @@ int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t
   p.h_k = h->h_k;
   p.g = h->g;
   p.L_max = h->max_seq_len;
-  p.N = N;
+  p.N = n_target;
   p.cand_cap = kTopnCap;
   p.scale = h->scale;
   p.samp = h->samp;
   p.t_lo = h->t_lo;
+  p.m_ref = ref ? h->m_ref : nullptr;
   const dim3 sgrid(h->batch * h->h_k, kSampleParts);
   const size_t smem = static_cast<size_t>(h->g) * h->d * sizeof(float);
   cudaError_t e = (h->d == 64)
@@ -231,7 +254,8 @@ int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t
 
 // S2-S4 from the candidate lists (a programmatic dependent of the score pass).
 int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
-                const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_logit, void* out) {
+                const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_logit, void* out,
+                int mode, float* log_tau) {
   TopnParams p;
   p.cand_mask = h->cand_mask;
   p.mask_stride = h->mask_stride;
@@ -245,6 +269,12 @@ int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   p.g_v = h->g_v;
   p.L_max = h->max_seq_len;
   p.N = N;
+  p.cap = mode == kModeStep ? 2 * N : N;
+  p.cand_cap = kTopnCap;
+  p.lse_part = h->lse_part;
+  p.m_ref = h->m_ref;
+  p.t_lo = h->t_lo;
+  p.log_tau = log_tau;
   p.sel_idx = sel_idx;
   p.sel_logit = sel_logit;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -254,9 +284,21 @@ int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = h->status;
   const dim3 grid(h->batch * h->h_q);
-  const cudaError_t e = (h->d == 64)
-      ? launch(h, topn_kernel<64>, grid, dim3(kTopnThreads), kTopnSmemBytes, kPdl, p)
-      : launch(h, topn_kernel<128>, grid, dim3(kTopnThreads), kTopnSmemBytes, kPdl, p);
+  const dim3 block(kTopnThreads);
+  constexpr size_t narrow = TopnLayout<kTopnSelNarrow>::kBytes, wide = TopnLayout<kTopnSelMax>::kBytes;
+  cudaError_t e;
+  if (mode == kModeExact)
+    e = (h->d == 64) ? launch(h, topn_kernel<64, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
+                     : launch(h, topn_kernel<128, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p);
+  else if (mode == kModeCalibrate)
+    e = (h->d == 64) ? launch(h, topn_kernel<64, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
+                     : launch(h, topn_kernel<128, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p);
+  else if (p.cap <= kTopnSelNarrow)
+    e = (h->d == 64) ? launch(h, topn_kernel<64, kModeStep, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
+                     : launch(h, topn_kernel<128, kModeStep, kTopnSelNarrow>, grid, block, narrow, kPdl, p);
+  else
+    e = (h->d == 64) ? launch(h, topn_kernel<64, kModeStep, kTopnSelMax>, grid, block, wide, kPdl, p)
+                     : launch(h, topn_kernel<128, kModeStep, kTopnSelMax>, grid, block, wide, kPdl, p);
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
@@ -342,15 +384,22 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // selection from candidates -> gather) needs the candidate lists and a selection small
 // enough for them; otherwise every score goes through the score workspace.
 bool use_candidates(const saga_ctx* h, int N) {
-  return h->cand_mask != nullptr && N <= kTopnSelMax && N <= kTopnCap / 4 && h->d <= kTopnMaxD &&
+  return h->cand_mask != nullptr && N <= kTopnSelNarrow && N <= kTopnCap / 4 && h->d <= kTopnMaxD &&
          (N < h->max_seq_len || h->max_seq_len <= kTopnCap);
 }
 
+// mode: kModeExact (the decode step), kModeCalibrate (also writes log_tau) or
+// kModeStep (selects with log_tau; selection rows of width 2N).
 int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
-                const int32_t* seq_lens, int N, void* out, int32_t* sel_idx, float* sel_logit) {
+                const int32_t* seq_lens, int N, void* out, int32_t* sel_idx, float* sel_logit,
+                int mode = kModeExact, float* log_tau = nullptr) {
   if (!q || !k_cache || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
+  if (mode != kModeExact) {
+    if (!log_tau) return SAGA_ERR_INVALID_ARG;
+    if (!use_candidates(h, N) || 2 * N > kTopnSelMax) return SAGA_ERR_UNSUPPORTED;
+  }
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
   const bool prof = h->prof && h->prof_n < h->prof_max;
@@ -362,11 +411,14 @@ int decode_impl(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   if (prof && record_event(ev[0], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
   int rc;
   if (use_candidates(h, N)) {
-    if ((rc = launch_bounds(h, q, k_cache, seq_lens, N))) return rc;
+    // a step keeps up to 2N entries: its candidates cover the 2N largest scores
+    const int n_target = mode == kModeStep ? 2 * N : N;
+    const bool lse = mode != kModeExact;
+    if ((rc = launch_bounds(h, q, k_cache, seq_lens, n_target, lse))) return rc;
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
-    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true))) return rc;
+    if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true, lse))) return rc;
     if (prof && record_event(ev[2], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
-    if ((rc = launch_topn(h, q, k_cache, v_cache, seq_lens, N, si, sl, out))) return rc;
+    if ((rc = launch_topn(h, q, k_cache, v_cache, seq_lens, N, si, sl, out, mode, log_tau))) return rc;
   } else {
     if (prof && record_event(ev[1], h->stream) != cudaSuccess) return SAGA_ERR_CUDA;
     if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, true))) return rc;
@@ -435,7 +487,7 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   const size_t rows = static_cast<size_t>(max_batch) * h_q;
   const size_t z_bytes = rows * h->z_stride * sizeof(float);
   const size_t stat_bytes = rows * sizeof(uint32_t);
-  const size_t sel_bytes = rows * static_cast<size_t>(max_N) * 4;
+  const size_t sel_bytes = rows * static_cast<size_t>(max_N) * 2 * 4;   // a step keeps up to 2N
   const size_t qo_bytes = rows * head_dim * 2;
   const int slots = max_N < max_seq_len ? max_N : max_seq_len;
   h->max_chunks = (slots + kGatherRows - 1) / kGatherRows;
@@ -447,7 +499,8 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   const size_t samp_bytes = rows * static_cast<size_t>(kSampleSize) * 4;
   const size_t total = al(z_bytes) + 2 * al(stat_bytes) + 2 * al(sel_bytes) + al(256) +
                        2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4) +
-                       al(part_bytes) + 2 * al(stat_bytes) + al(mask_bytes) + al(samp_bytes);
+                       al(part_bytes) + 2 * al(stat_bytes) + al(mask_bytes) + al(samp_bytes) +
+                       al(stat_bytes) + al(mask_bytes);
   if (cudaMalloc(&h->ws, total) != cudaSuccess) { delete h; return SAGA_ERR_CUDA; }
   uint8_t* w = static_cast<uint8_t*>(h->ws);
   h->z = reinterpret_cast<float*>(w); w += al(z_bytes);
@@ -463,7 +516,9 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->counter = reinterpret_cast<uint32_t*>(w); w += al(stat_bytes);
   h->cand_mask = reinterpret_cast<uint32_t*>(w); w += al(mask_bytes);
   h->samp = reinterpret_cast<float*>(w); w += al(samp_bytes);
-  h->t_lo = reinterpret_cast<float*>(w);
+  h->t_lo = reinterpret_cast<float*>(w); w += al(stat_bytes);
+  h->m_ref = reinterpret_cast<float*>(w); w += al(stat_bytes);
+  h->lse_part = reinterpret_cast<float*>(w);
   h->scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
   if (cudaMemset(h->stat_min, 0xFF, stat_bytes) != cudaSuccess ||
       cudaMemset(h->counter, 0x00, stat_bytes) != cudaSuccess ||
@@ -503,6 +558,24 @@ int saga_decode_attn_ex(saga_handle h, const void* q, const void* k_cache, const
   if (!h) return SAGA_ERR_INVALID_ARG;
   if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
   return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit);
+}
+
+int saga_atopn_calibrate(saga_handle h, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* seq_lens, int h_q, int h_k, int h_v, int head_dim, int N,
+                         void* out, int32_t* sel_idx, float* sel_logit, float* log_tau) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit, kModeCalibrate,
+                     log_tau);
+}
+
+int saga_atopn_step(saga_handle h, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* seq_lens, int h_q, int h_k, int h_v, int head_dim, int N,
+                    const float* log_tau, void* out, int32_t* sel_idx, float* sel_logit) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit, kModeStep,
+                     const_cast<float*>(log_tau));
 }
 
 int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache,

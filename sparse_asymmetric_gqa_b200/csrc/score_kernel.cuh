@@ -22,6 +22,13 @@
 //     back at once), for larger groups each takes half of the heads.  They
 //     scale, and either store z row-wise (coalesced per head) with per-(b, j)
 //     min/max statistics, or append the candidates of the selector.
+//
+// With kLse (candidate mode), the epilogue also writes, per query head
+// and 32-position chunk, the sum of exp(z - m_ref[row]) over the chunk's
+// positions: the pieces of the row's log-sum-exp, from which a calibrated
+// probability threshold becomes a logit threshold ("More Value per Key",
+// App. C.1).  A term whose exponent exceeds kLseMaxExp makes the chunk's sum
+// +inf, which sends the row to the selector's exact fallback.
 #pragma once
 
 #include <cuda.h>
@@ -33,6 +40,8 @@ constexpr int kTileM = 128;          // positions per tile (MMA M)
 constexpr int kEpiWarps = 8;         // two per TMEM lane quarter
 constexpr int kScoreThreads = 64 + 32 * kEpiWarps;   // TMA, MMA, epilogue warps
 constexpr int kMaxBatch = 1024;
+// Largest exponent z - m_ref summed: a row of up to 2^24 terms stays below 2^24 e^64 < FLT_MAX.
+constexpr float kLseMaxExp = 64.0f;
 
 struct ScoreParams {
   const int32_t* seq_lens;   // [B]
@@ -41,6 +50,8 @@ struct ScoreParams {
   uint32_t* cand_mask;       // [B*h_q][mask_stride]: bit i of word c = position 32c + i passed
   long long mask_stride;
   const float* t_lo;         // [B*h_q] candidate bounds, written by the preceding kernel
+  const float* m_ref;        // [B*h_q] exp-sum references (+inf: no sums), with lse_part
+  float* lse_part;           // [B*h_q][mask_stride] per-chunk sums of exp(z - m_ref) (kLse)
   uint32_t* stat_min;        // [B*h_q] ordered keys, or nullptr
   uint32_t* stat_max;
   int* status;
@@ -114,6 +125,33 @@ __device__ __forceinline__ void st_global_hint(uint32_t* p, uint32_t v, uint64_t
   asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" :: "l"(p), "r"(v), "l"(pol) : "memory");
 }
 
+// Sums across the warp of each of the H values of every lane (a butterfly that
+// halves the values held per lane at each step: 16 or 31 shuffles for all H).
+// Returns, in lane l, the sum for value l / (32 / HP), HP = H rounded up to 16
+// or 32; a fixed order of additions, so the result is reproducible.
+template <int H>
+__device__ __forceinline__ float warp_transpose_sum(const float (&v)[H], int lane) {
+  constexpr int HP = H <= 16 ? 16 : 32;
+  static_assert(H <= 32, "at most 32 values per lane");
+  float w[HP];
+#pragma unroll
+  for (int i = 0; i < HP; ++i) w[i] = i < H ? v[i] : 0.0f;
+#pragma unroll
+  for (int c = HP; c > 1; c >>= 1) {
+    const int o = HP == 32 ? c / 2 : c;        // the lane bit that picks the half kept
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < c / 2; ++i) {
+      const float send = up ? w[i] : w[i + c / 2];
+      const float keep = up ? w[i + c / 2] : w[i];
+      w[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float r = w[0];
+  if (HP == 16) r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
   *abort_flag = 1;
   atomicOr(status, 0x2 /* SAGA_STATUS_TIMEOUT */);
@@ -128,7 +166,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // goes to cand_mask[row][c] and their order-preserving keys, in position
 // order, to the row's z slots [32c, 32c + popcount).  No atomics on the data
 // path: every chunk has its own slots.
-template <int D, int NPAD, bool kCand>
+// kLse (candidate mode only): the chunk sums of exp(z - m_ref) go to lse_part.
+template <int D, int NPAD, bool kCand, bool kLse = false>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_kernel(const __grid_constant__ CUtensorMap tmap_k,
              const __grid_constant__ CUtensorMap tmap_q, const ScoreParams p) {
@@ -325,9 +364,11 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         rmax[e] = 0u;
       }
     };
-    float tl[H];
+    float tl[H], mr[H];
 #pragma unroll
-    for (int e = 0; e < H; ++e) tl[e] = INFINITY;
+    for (int e = 0; e < H; ++e) { tl[e] = INFINITY; mr[e] = INFINITY; }
+    static_assert(kCand || !kLse, "chunk sums come with the candidate mode");
+    constexpr bool lse = kLse;
     if (n_tiles > 0) {
       TileCursor c;
       c.seek(u0, unit_off, lens, p.B, p.h_k);
@@ -342,6 +383,10 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int rowg = c.b * p.h_q + c.kh * p.g + h0;
 #pragma unroll
             for (int e = 0; e < H; ++e) tl[e] = (h0 + e < p.g) ? __ldcg(p.t_lo + rowg + e) : INFINITY;
+            if (lse) {
+#pragma unroll
+              for (int e = 0; e < H; ++e) mr[e] = (h0 + e < p.g) ? __ldcg(p.m_ref + rowg + e) : INFINITY;
+            }
           }
         }
         float acc[H];
@@ -354,10 +399,15 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int chunk = c.t * (kTileM / 32) + quad;
           uint32_t* kslot = reinterpret_cast<uint32_t*>(p.z) + static_cast<long long>(row0) * p.z_stride + chunk * 32;
           uint32_t my_m = 0u;
+          float ex[H];
 #pragma unroll
           for (int e = 0; e < H; ++e) {
             // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
             const float zz = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
+            if (lse) {   // exp(-inf) = 0 for rows without a reference
+              const float a = zz - mr[e];
+              ex[e] = (valid && h0 + e < p.g) ? (a > kLseMaxExp ? INFINITY : expf(a)) : 0.0f;
+            }
             const bool take = valid && h0 + e < p.g && zz >= tl[e];
             const uint32_t m = __ballot_sync(0xffffffffu, take);
             if (lane == e) my_m = m;
@@ -367,6 +417,13 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           if (lane < H && h0 + lane < p.g && chunk * 32 < c.Lb)   // lane e: head e's mask
             st_global_hint(p.cand_mask + static_cast<long long>(row0 + lane) * p.mask_stride + chunk, my_m, pol_z);
+          if (lse) {
+            constexpr int kSpread = H <= 16 ? 2 : 1;             // lanes per head in the result
+            const float sum = warp_transpose_sum<H>(ex, lane);
+            const int e = lane / kSpread;
+            if (lane % kSpread == 0 && e < H && h0 + e < p.g && chunk * 32 < c.Lb)
+              st_global_hint(p.lse_part + static_cast<long long>(row0 + e) * p.mask_stride + chunk, sum, pol_z);
+          }
         } else if (valid) {
           float* zrow = p.z + static_cast<long long>(row0) * p.z_stride + pos;
 #pragma unroll

@@ -47,7 +47,8 @@ namespace saga {
 constexpr int kTopnThreads = 256;
 constexpr int kTopnWarps = kTopnThreads / 32;
 constexpr int kTopnCap = 8192;                    // candidates held in shared memory
-constexpr int kTopnSelMax = 2048;                 // largest N of the candidate path
+constexpr int kTopnSelMax = 4096;                 // widest selection list (2N of a step)
+constexpr int kTopnSelNarrow = 2048;              // selection lists of the exact path (N)
 constexpr int kTopnBins = 2048;                   // 11-bit radix digits
 constexpr int kTopnBinsPer = kTopnBins / kTopnThreads;   // digits owned by a thread in a scan
 constexpr int kTopnPer = 16;                      // entries per thread per step of the ordered pass
@@ -56,20 +57,32 @@ constexpr int kTopnRound = 4;                     // chunks per thread per round
 constexpr int kTopnMaxRun = 8;                    // chunks per thread on the shared-memory path
 constexpr int kTopnMaxD = 128;
 
-// Dynamic shared memory, in 32-bit words; every region starts on a 16-byte boundary.
-constexpr int kTopnOffKey = 0;                                  // [kTopnCap] candidate keys
-constexpr int kTopnOffPos = kTopnOffKey + kTopnCap;             // [kTopnCap] candidate positions
-constexpr int kTopnOffSelPos = kTopnOffPos + kTopnCap;          // [kTopnSelMax] selected positions
-constexpr int kTopnOffSelW = kTopnOffSelPos + kTopnSelMax;      // [kTopnSelMax] softmax weights
-constexpr int kTopnOffHist = kTopnOffSelW + kTopnSelMax;        // [kTopnBins]; P.V partials [warps][D]
-constexpr int kTopnOffScan = kTopnOffHist + kTopnBins;          // [kTopnWarps]
-constexpr int kTopnOffMisc = kTopnOffScan + kTopnWarps;         // [8]
-constexpr int kTopnSmemWords = kTopnOffMisc + 8;
-constexpr size_t kTopnSmemBytes = sizeof(uint32_t) * kTopnSmemWords;
-static_assert(kTopnOffPos % 4 == 0 && kTopnOffSelPos % 4 == 0 && kTopnOffSelW % 4 == 0 &&
-              kTopnOffHist % 4 == 0 && kTopnOffScan % 4 == 0 && kTopnOffMisc % 4 == 0,
-              "shared regions on 16-byte boundaries");
+// Dynamic shared memory, in 32-bit words, for selection lists of up to kSel
+// entries; every region starts on a 16-byte boundary.  (90 KB for kSel = 2048:
+// two CTAs per SM; the wide layout of a step with N > 1024 takes 106 KB.)
+template <int kSel>
+struct TopnLayout {
+  static constexpr int kOffKey = 0;                             // [kTopnCap] candidate keys
+  static constexpr int kOffPos = kOffKey + kTopnCap;            // [kTopnCap] candidate positions
+  static constexpr int kOffSelPos = kOffPos + kTopnCap;         // [kSel] selected positions
+  static constexpr int kOffSelW = kOffSelPos + kSel;            // [kSel] softmax weights
+  static constexpr int kOffHist = kOffSelW + kSel;              // [kTopnBins]; P.V partials [warps][D]
+  static constexpr int kOffScan = kOffHist + kTopnBins;         // [kTopnWarps]
+  static constexpr int kOffMisc = kOffScan + kTopnWarps;        // [8]
+  static constexpr int kWords = kOffMisc + 8;
+  static constexpr size_t kBytes = sizeof(uint32_t) * kWords;
+  static_assert(kOffPos % 4 == 0 && kOffSelPos % 4 == 0 && kOffSelW % 4 == 0 &&
+                kOffHist % 4 == 0 && kOffScan % 4 == 0 && kOffMisc % 4 == 0,
+                "shared regions on 16-byte boundaries");
+};
 static_assert(kTopnWarps * kTopnMaxD <= kTopnBins, "P.V partials fit the histogram region");
+
+// What a call selects.  kModeExact: the top N.  kModeCalibrate: the top N, and
+// log tau = z_(N_b) - logsumexp(z), the log-probability of the N_b-th largest
+// score, per row.  kModeStep: every score z >= log tau + logsumexp(z) for the
+// row's calibrated log tau, in ascending position order, the first cap = 2N
+// kept ("More Value per Key", App. C.1).
+enum TopnMode { kModeExact = 0, kModeCalibrate = 1, kModeStep = 2 };
 
 struct TopnParams {
   const uint32_t* cand_mask;    // [B*h_q][mask_stride] passing positions per 32-position chunk
@@ -78,8 +91,14 @@ struct TopnParams {
   long long z_stride;
   const int32_t* seq_lens;      // [B]
   int h_q, h_k, g, h_v, g_v, L_max, N;
-  int32_t* sel_idx;             // [B*h_q][N]
-  float* sel_logit;             // [B*h_q][N]
+  int cap;                      // width of a selection list row: N, or 2N in step mode
+  int cand_cap;                 // rows with L <= cand_cap: every position is a candidate
+  const float* lse_part;        // [B*h_q][mask_stride] chunk sums of exp(z - m_ref) (modes 1, 2)
+  const float* m_ref;           // [B*h_q] their reference
+  const float* t_lo;            // [B*h_q] the candidates' bound (step mode checks t >= t_lo)
+  float* log_tau;               // [B*h_q] written by calibration, read by a step
+  int32_t* sel_idx;             // [B*h_q][cap]
+  float* sel_logit;             // [B*h_q][cap]
   const __nv_bfloat16* q;       // [B][h_q][D] (scoring a row again, fallback)
   const __nv_bfloat16* k_cache; // [B][h_k][L_max][D]
   const __nv_bfloat16* v_cache; // [B][h_v][L_max][D]
@@ -299,6 +318,87 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Block-wide sum and max, every thread the same result (a fixed order of operations).
+__device__ __forceinline__ float topn_block_sum(float v, uint32_t* s_scan) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* s = reinterpret_cast<float*>(s_scan);
+  v = warp_sum(v);
+  if (lane == 0) s[warp] = v;
+  __syncthreads();
+  float t = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kTopnWarps; ++w) t += s[w];
+  __syncthreads();
+  return t;
+}
+__device__ __forceinline__ uint32_t topn_block_max(uint32_t v, uint32_t* s_scan) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = __reduce_max_sync(0xffffffffu, v);
+  if (lane == 0) s_scan[warp] = v;
+  __syncthreads();
+  uint32_t t = 0u;
+#pragma unroll
+  for (int w = 0; w < kTopnWarps; ++w) t = max(t, s_scan[w]);
+  __syncthreads();
+  return t;
+}
+
+// logsumexp of the n entries of src (a whole row): max, then the sum of exp(z - max).
+template <class Src>
+__device__ float topn_lse(const Src& src, int n, uint32_t* s_scan) {
+  uint32_t hi = 0u;
+  for (int i = threadIdx.x; i < n; i += kTopnThreads) {
+    uint32_t key;
+    if (src.get(i, key)) hi = max(hi, key);
+  }
+  const float m = key_to_float(topn_block_max(hi, s_scan));
+  float sum = 0.0f;
+  for (int i = threadIdx.x; i < n; i += kTopnThreads) {
+    uint32_t key;
+    if (src.get(i, key)) sum += expf(key_to_float(key) - m);
+  }
+  return m + logf(topn_block_sum(sum, s_scan));
+}
+
+// Step selection: every entry with key >= kt, visited in ascending position
+// order, the first cap kept; a kept entry's slot is the count of passing
+// entries before it (one block scan per step of kTopnStep entries).  Writes the
+// caller's lists and, in shared memory, the positions and logits; returns how
+// many entries were kept (every thread the same).
+template <class Src>
+__device__ uint32_t topn_emit_ge(const Src& src, int n, uint32_t kt, uint32_t cap, int32_t* idx_out,
+                                 float* logit_out, int32_t* s_selpos, float* s_selz, uint32_t* s_scan) {
+  uint32_t done = 0u;
+  for (int base = 0; base < n && done < cap; base += kTopnStep) {
+    const int i0 = base + kTopnPer * static_cast<int>(threadIdx.x);
+    uint32_t key[kTopnPer];
+    bool val[kTopnPer];
+    uint32_t nge = 0u;
+#pragma unroll
+    for (int e = 0; e < kTopnPer; ++e) {
+      val[e] = src.get(i0 + e, key[e]) && key[e] >= kt;
+      nge += val[e] ? 1u : 0u;
+    }
+    uint32_t tot;
+    uint32_t slot = done + topn_excl_scan(nge, s_scan, tot);
+#pragma unroll
+    for (int e = 0; e < kTopnPer; ++e) {
+      if (!val[e]) continue;
+      if (slot < cap) {
+        const int pos = src.position(i0 + e);
+        const float z = key_to_float(key[e]);
+        idx_out[slot] = pos;
+        logit_out[slot] = z;
+        s_selpos[slot] = pos;
+        s_selz[slot] = z;
+      }
+      ++slot;
+    }
+    done += tot;
+  }
+  return min(done, cap);
+}
+
 // Keys of one row scored on CUDA cores: key(fl(fl(q . k_i) * scale)), -0 -> +0.
 template <int D>
 __device__ void topn_rescore(const __nv_bfloat16* q, const __nv_bfloat16* keys, int L, float scale,
@@ -323,18 +423,20 @@ __device__ void topn_rescore(const __nv_bfloat16* q, const __nv_bfloat16* keys, 
   }
 }
 
-template <int D>
+// kMode: a TopnMode; kSel: the layout's selection capacity (>= the list width p.cap).
+template <int D, int kMode, int kSel>
 __global__ void __launch_bounds__(kTopnThreads, 2)
 topn_kernel(const TopnParams p) {
+  using Lay = TopnLayout<kSel>;
   extern __shared__ __align__(16) uint32_t topn_smem[];
-  uint32_t* s_key = topn_smem + kTopnOffKey;
-  int32_t* s_pos = reinterpret_cast<int32_t*>(topn_smem + kTopnOffPos);
-  int32_t* s_selpos = reinterpret_cast<int32_t*>(topn_smem + kTopnOffSelPos);
-  float* s_selw = reinterpret_cast<float*>(topn_smem + kTopnOffSelW);
-  uint32_t* s_hist = topn_smem + kTopnOffHist;
-  float* s_part = reinterpret_cast<float*>(topn_smem + kTopnOffHist);   // after the selection
-  uint32_t* s_scan = topn_smem + kTopnOffScan;
-  uint32_t* s_misc = topn_smem + kTopnOffMisc;
+  uint32_t* s_key = topn_smem + Lay::kOffKey;
+  int32_t* s_pos = reinterpret_cast<int32_t*>(topn_smem + Lay::kOffPos);
+  int32_t* s_selpos = reinterpret_cast<int32_t*>(topn_smem + Lay::kOffSelPos);
+  float* s_selw = reinterpret_cast<float*>(topn_smem + Lay::kOffSelW);
+  uint32_t* s_hist = topn_smem + Lay::kOffHist;
+  float* s_part = reinterpret_cast<float*>(topn_smem + Lay::kOffHist);   // after the selection
+  uint32_t* s_scan = topn_smem + Lay::kOffScan;
+  uint32_t* s_misc = topn_smem + Lay::kOffMisc;
 
   pdl_wait();                                    // the candidate lists are complete
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -342,29 +444,42 @@ topn_kernel(const TopnParams p) {
   const int b = bj / p.h_q, j = bj % p.h_q;
   const int L = p.seq_lens[b];
   const int N = p.N;
-  int32_t* idx_out = p.sel_idx + static_cast<long long>(bj) * N;
-  float* logit_out = p.sel_logit + static_cast<long long>(bj) * N;
+  constexpr int mode = kMode;
+  const int cap = p.cap;
+  int32_t* idx_out = p.sel_idx + static_cast<long long>(bj) * cap;
+  float* logit_out = p.sel_logit + static_cast<long long>(bj) * cap;
   __nv_bfloat16* orow = p.out + static_cast<long long>(bj) * D;
   if (L < 1 || L > p.L_max) {                    // invalid row: padding and a zero output
-    if (tid == 0) atomicOr(p.status, 0x1 /* SAGA_STATUS_BAD_SEQ_LEN */);
-    for (int r = tid; r < N; r += kTopnThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
+    if (tid == 0) {
+      atomicOr(p.status, 0x1 /* SAGA_STATUS_BAD_SEQ_LEN */);
+      if (mode == kModeCalibrate) p.log_tau[bj] = -INFINITY;
+    }
+    for (int r = tid; r < cap; r += kTopnThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
     for (int e = tid; e < D; e += kTopnThreads) orow[e] = __float2bfloat16_rn(0.0f);
     return;
   }
-  const uint32_t n_b = static_cast<uint32_t>(N < L ? N : L);
   const uint32_t* mrow = p.cand_mask + static_cast<long long>(bj) * p.mask_stride;
   uint32_t* krow = p.zkey + static_cast<long long>(bj) * p.z_stride;
   const int nch = (L + 31) / 32;
+  // the row's log-sum-exp comes from the score pass's chunk sums when the row
+  // has a sampled reference (L > cand_cap), else from its complete candidate list
+  const bool sums = mode != kModeExact && L > p.cand_cap;
+  const float* lrow = sums ? p.lse_part + static_cast<long long>(bj) * p.mask_stride : nullptr;
 
   // ---- candidate count and each chunk run's offset: thread t owns chunks [c0, c1);
   // the first round also loads the first key sector of its first kTopnRound chunks
+  // (and the chunk sums)
   const int cpt = (nch + kTopnThreads - 1) / kTopnThreads;
   const int c0 = min(nch, tid * cpt), c1 = min(nch, c0 + cpt);
   const bool fits = cpt <= kTopnMaxRun;
   uint32_t run_mask[kTopnMaxRun];
+  float run_sum[kTopnMaxRun];
   uint4 sec[kTopnRound][2];
 #pragma unroll
-  for (int u = 0; u < kTopnMaxRun; ++u) run_mask[u] = (c0 + u < c1) ? __ldcg(mrow + c0 + u) : 0u;
+  for (int u = 0; u < kTopnMaxRun; ++u) {
+    run_mask[u] = (c0 + u < c1) ? __ldcg(mrow + c0 + u) : 0u;
+    run_sum[u] = (sums && c0 + u < c1) ? __ldcg(lrow + c0 + u) : 0.0f;
+  }
 #pragma unroll
   for (int u = 0; u < kTopnRound; ++u) {
     const uint4* kp = reinterpret_cast<const uint4*>(krow + (c0 + u) * 32);
@@ -372,18 +487,28 @@ topn_kernel(const TopnParams p) {
     sec[u][1] = (c0 + u < c1) ? __ldcg(kp + 1) : make_uint4(0u, 0u, 0u, 0u);
   }
   uint32_t cnt = 0u;
+  float lsum = 0.0f;
 #pragma unroll
-  for (int u = 0; u < kTopnMaxRun; ++u) cnt += __popc(run_mask[u]);
+  for (int u = 0; u < kTopnMaxRun; ++u) { cnt += __popc(run_mask[u]); lsum += run_sum[u]; }
   if (!fits)
-    for (int c = c0 + kTopnMaxRun; c < c1; ++c) cnt += __popc(__ldcg(mrow + c));
+    for (int c = c0 + kTopnMaxRun; c < c1; ++c) {
+      cnt += __popc(__ldcg(mrow + c));
+      if (sums) lsum += __ldcg(lrow + c);
+    }
   uint32_t C;
   const uint32_t off = topn_excl_scan(cnt, s_scan, C);
+  float lse = 0.0f;
+  bool lse_ok = false;
+  if (sums) {
+    const float S = topn_block_sum(lsum, s_scan);
+    const float mref = __ldcg(p.m_ref + bj);
+    lse_ok = S > 0.0f && S <= 3.402823466e38f && mref > -INFINITY && mref < INFINITY;
+    lse = mref + logf(S);
+  }
 
-  uint32_t need, kmax;
-  float wsum;
-  if (C >= n_b && C <= static_cast<uint32_t>(kTopnCap) && fits) {
-    // Each chunk's keys are contiguous at its slots, in position order: write
-    // them with the positions of the mask bits.
+  // Each chunk's keys are contiguous at its slots, in position order: write
+  // them to shared memory with the positions of the mask bits.
+  auto gather_list = [&]() {
     uint32_t o = off;
 #pragma unroll
     for (int u0 = 0; u0 < kTopnMaxRun; u0 += kTopnRound) {
@@ -421,25 +546,77 @@ topn_kernel(const TopnParams p) {
       }
     }
     __syncthreads();
-    const TopnListSrc src{s_key, s_pos, static_cast<int>(C)};
-    const uint32_t T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need, &kmax);
-    wsum = topn_emit(src, src.n, T, need, n_b, key_to_float(kmax), idx_out, logit_out, s_selpos,
-                     s_selw, s_scan);
-  } else {
+  };
+  // The row scored again on CUDA cores (the candidates do not cover what is selected).
+  auto rescore = [&]() {
     if (tid == 0) atomicOr(p.status, 0x200 /* SAGA_STATUS_INFO_ROBUST_PATH */);
-    const bool all = C < n_b;                    // the bound missed: score the row again
-    if (all) {
-      const __nv_bfloat16* keys =
-          p.k_cache + (static_cast<long long>(b) * p.h_k + j / p.g) * p.L_max * D;
-      topn_rescore<D>(p.q + static_cast<long long>(bj) * D, keys, L, p.scale, krow);
-      __syncthreads();                           // the row's keys are visible to the whole CTA
+    const __nv_bfloat16* keys =
+        p.k_cache + (static_cast<long long>(b) * p.h_k + j / p.g) * p.L_max * D;
+    topn_rescore<D>(p.q + static_cast<long long>(bj) * D, keys, L, p.scale, krow);
+    __syncthreads();                             // the row's keys are visible to the whole CTA
+  };
+
+  uint32_t n_out;                                // entries of the selection
+  float wsum = 0.0f;
+  if (mode != kModeStep) {
+    const uint32_t n_b = static_cast<uint32_t>(N < L ? N : L);
+    uint32_t need, kmax, T;
+    const bool all = C < n_b || (sums && !lse_ok);
+    if (!all && C <= static_cast<uint32_t>(kTopnCap) && fits) {
+      gather_list();
+      const TopnListSrc src{s_key, s_pos, static_cast<int>(C)};
+      T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need, &kmax);
+      wsum = topn_emit(src, src.n, T, need, n_b, key_to_float(kmax), idx_out, logit_out, s_selpos,
+                       s_selw, s_scan);
+      if (mode == kModeCalibrate && !sums) lse = topn_lse(src, src.n, s_scan);
+    } else {
+      // a list longer than kTopnCap is selected from the slots in global memory;
+      // a list shorter than N_b (the sampled bound missed) has the row scored again
+      if (all) rescore();
+      else if (tid == 0) atomicOr(p.status, 0x200 /* SAGA_STATUS_INFO_ROBUST_PATH */);
+      const TopnSlotSrc src{mrow, krow, all ? L : nch * 32, all};
+      T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need, &kmax);
+      wsum = topn_emit(src, src.n, T, need, n_b, key_to_float(kmax), idx_out, logit_out, s_selpos,
+                       s_selw, s_scan);
+      if (mode == kModeCalibrate && !(sums && lse_ok)) lse = topn_lse(src, src.n, s_scan);
     }
-    const TopnSlotSrc src{mrow, krow, all ? L : nch * 32, all};
-    const uint32_t T = topn_radix(src, src.n, n_b, s_hist, s_scan, s_misc, &need, &kmax);
-    wsum = topn_emit(src, src.n, T, need, n_b, key_to_float(kmax), idx_out, logit_out, s_selpos,
-                     s_selw, s_scan);
+    if (mode == kModeCalibrate && tid == 0) p.log_tau[bj] = key_to_float(T) - lse;
+    n_out = n_b;
+  } else {
+    float lt = __ldcg(p.log_tau + bj);
+    if (lt != lt) lt = -INFINITY;                // NaN: no threshold
+    float t = lt + lse;
+    const bool miss = sums && (!lse_ok || !(t >= __ldcg(p.t_lo + bj)));
+    auto threshold_key = [&]() { return ordered_key(__fadd_rn(t, 0.0f)); };
+    if (!miss && C <= static_cast<uint32_t>(kTopnCap) && fits) {
+      gather_list();
+      const TopnListSrc src{s_key, s_pos, static_cast<int>(C)};
+      if (!sums) t = lt + topn_lse(src, src.n, s_scan);
+      n_out = topn_emit_ge(src, src.n, threshold_key(), static_cast<uint32_t>(cap), idx_out,
+                           logit_out, s_selpos, s_selw, s_scan);
+    } else {
+      if (miss) rescore();
+      else if (tid == 0) atomicOr(p.status, 0x200 /* SAGA_STATUS_INFO_ROBUST_PATH */);
+      const TopnSlotSrc src{mrow, krow, miss ? L : nch * 32, miss};
+      if (!sums || !lse_ok) t = lt + topn_lse(src, src.n, s_scan);
+      n_out = topn_emit_ge(src, src.n, threshold_key(), static_cast<uint32_t>(cap), idx_out,
+                           logit_out, s_selpos, s_selw, s_scan);
+    }
+    // softmax weights exp(z - max) over the kept logits, in place of them
+    __syncthreads();
+    uint32_t hi = 0u;
+    for (uint32_t i = tid; i < n_out; i += kTopnThreads) hi = max(hi, ordered_key(s_selw[i]));
+    const float zmax = key_to_float(topn_block_max(hi, s_scan));
+    for (uint32_t i = tid; i < n_out; i += kTopnThreads) {
+      const float w = expf(s_selw[i] - zmax);
+      s_selw[i] = w;
+      wsum += w;
+    }
   }
-  for (int r = static_cast<int>(n_b) + tid; r < N; r += kTopnThreads) { idx_out[r] = -1; logit_out[r] = -INFINITY; }
+  for (int r = static_cast<int>(n_out) + tid; r < cap; r += kTopnThreads) {
+    idx_out[r] = -1;
+    logit_out[r] = -INFINITY;
+  }
 
   // ---- softmax denominator
   wsum = warp_sum(wsum);
@@ -456,20 +633,20 @@ topn_kernel(const TopnParams p) {
   float acc[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) acc[e] = 0.0f;
-  for (int g0 = warp * 32; g0 < static_cast<int>(n_b); g0 += kTopnWarps * 32) {
+  for (int g0 = warp * 32; g0 < static_cast<int>(n_out); g0 += kTopnWarps * 32) {
     if constexpr (EPL == 4) {
       uint2 raw[32];
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         const int sl = g0 + u;
-        raw[u] = sl < static_cast<int>(n_b)
+        raw[u] = sl < static_cast<int>(n_out)
                      ? __ldg(reinterpret_cast<const uint2*>(vbase + static_cast<long long>(s_selpos[sl]) * D))
                      : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         const int sl = g0 + u;
-        const float wu = sl < static_cast<int>(n_b) ? s_selw[sl] : 0.0f;
+        const float wu = sl < static_cast<int>(n_out) ? s_selw[sl] : 0.0f;
         const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u].x));
         const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u].y));
         acc[0] = fmaf(wu, a.x, acc[0]);
@@ -482,14 +659,14 @@ topn_kernel(const TopnParams p) {
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         const int sl = g0 + u;
-        raw[u] = sl < static_cast<int>(n_b)
+        raw[u] = sl < static_cast<int>(n_out)
                      ? __ldg(reinterpret_cast<const uint32_t*>(vbase + static_cast<long long>(s_selpos[sl]) * D))
                      : 0u;
       }
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         const int sl = g0 + u;
-        const float wu = sl < static_cast<int>(n_b) ? s_selw[sl] : 0.0f;
+        const float wu = sl < static_cast<int>(n_out) ? s_selw[sl] : 0.0f;
         const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u]));
         acc[0] = fmaf(wu, a.x, acc[0]);
         acc[1] = fmaf(wu, a.y, acc[1]);

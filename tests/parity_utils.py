@@ -81,3 +81,101 @@ def check_row(gpu_idx, gpu_logit, gpu_out, q_row, k_rows, v_rows, N, what=""):
     out_on_gpu_set = oracle.combine(z_ref[sel], np.asarray(v_rows)[sel])
     assert_out_close(gpu_out, out_on_gpu_set, f"{what} out vs oracle on GPU set")
     return len(diff)
+
+
+# --------------------------------------------------------------------------- stateful Atop-N
+
+TAIL = 32          # the oracle's tail for m_hat (the threshold does not depend on it)
+EPS32 = 2.0 ** -24
+
+
+def lse_error(q_row, k_rows, z_ref, extra=0.0):
+    """The row's float64 log-sum-exp and a bound on the error of the GPU's fp32 one.
+
+    The GPU sums exp(z) of its fp32 scores: d(LSE)/dz_i = p_i, so the scores'
+    errors move it by at most sum_i p_i * bound_i; the sum itself (exp within
+    2 ulp, a reduction tree of depth < 32) adds 32 ulp relative, and the fp32
+    values of magnitude |LSE| and |extra| combined with it a few ulp each."""
+    m = z_ref.max()
+    e = np.exp(z_ref - m)
+    lse = m + math.log(e.sum())
+    p = e / e.sum()
+    err = float(p @ score_bound(q_row, k_rows)) + 32 * EPS32 + 8 * EPS32 * (abs(lse) + abs(extra))
+    return lse, err
+
+
+def check_log_tau(gpu_log_tau, q_row, k_rows, N, what=""):
+    """Calibration: log tau = z_(N_b) - logsumexp(z) of the row, against the oracle in
+    float64; tolerance: the N-th score within BAND plus its fp32 bound, and the
+    log-sum-exp's error bound."""
+    z_ref = oracle.scores(q_row, k_rows)
+    ref = math.log(oracle.calibrate_tau(z_ref, N))
+    n_b = min(N, z_ref.shape[0])
+    k = np.asarray(k_rows)
+    near = np.flatnonzero(np.abs(z_ref - np.sort(z_ref)[::-1][n_b - 1]) <= BAND)
+    _, err = lse_error(q_row, k_rows, z_ref, ref)
+    tol = BAND + float(score_bound(q_row, k[near]).max()) + err
+    assert abs(float(gpu_log_tau) - ref) <= tol, \
+        f"{what}: log tau {float(gpu_log_tau)} vs oracle {ref} (tolerance {tol})"
+
+
+def check_step_row(gpu_idx, gpu_logit, gpu_out, q_row, k_rows, v_rows, log_tau, N, what=""):
+    """A step of stateful Atop-N against the oracle replaying the same tau.
+
+    The oracle threshold is t = m_hat + log(tau * s_hat) in float64 with
+    tau = exp(log_tau) (the GPU's state).  The GPU keeps the positions with
+    z >= t in ascending order, at most 2N of them; a position may go either way
+    when its oracle score lies within BAND + its fp32 score bound + the bound
+    on the GPU threshold's error (its log-sum-exp, see lse_error) of t; the
+    output is compared with the
+    oracle's softmax and P.V over the GPU's kept set, and with the oracle's own
+    step output when the two sets agree.  Returns the number of kept
+    positions."""
+    z_ref = oracle.scores(q_row, k_rows)
+    L = z_ref.shape[0]
+    cap = 2 * N
+    tau = math.exp(float(log_tau))
+    t = oracle.step_threshold(z_ref, tau, TAIL)
+    gpu_idx = np.asarray(gpu_idx)
+    gpu_logit = np.asarray(gpu_logit, dtype=np.float64)
+    n = int((gpu_idx >= 0).sum())
+    sel = gpu_idx[:n]
+    assert (gpu_idx[n:] == -1).all(), f"{what}: padding"
+    assert np.isneginf(gpu_logit[n:]).all(), f"{what}: logit padding"
+    assert n <= cap
+    if n:
+        assert (np.diff(sel) > 0).all(), f"{what}: not strictly ascending"
+        assert sel.min() >= 0 and sel.max() < L, f"{what}: index out of range"
+    gpu_set = np.zeros(L, dtype=bool)
+    gpu_set[sel] = True
+    _, t_err = lse_error(q_row, k_rows, z_ref, abs(float(log_tau)) + abs(t))
+    band = BAND + t_err + score_bound(q_row, k_rows)
+    sure = z_ref > t + band
+    maybe = np.abs(z_ref - t) <= band
+    assert not (gpu_set & ~(sure | maybe)).any(), \
+        f"{what}: kept below the threshold {np.flatnonzero(gpu_set & ~(sure | maybe))[:5]}"
+    if (sure | maybe).sum() <= cap:
+        assert not (sure & ~gpu_set).any(), f"{what}: missed {np.flatnonzero(sure & ~gpu_set)[:5]}"
+    else:
+        # capacity binds: the first 2N passing positions, so every sure position
+        # before the last kept one is kept
+        assert n == cap, f"{what}: {n} kept, capacity {cap} binds"
+        early = sure & (np.arange(L) < sel[-1])
+        assert not (early & ~gpu_set).any(), f"{what}: skipped {np.flatnonzero(early & ~gpu_set)[:5]}"
+    if n:
+        bound = score_bound(q_row, np.asarray(k_rows)[sel])
+        err = np.abs(gpu_logit[:n] - z_ref[sel])
+        assert (err <= bound).all(), f"{what}: kept logits off by {err.max()}"
+        assert_out_close(gpu_out, oracle.combine(z_ref[sel], np.asarray(v_rows)[sel]),
+                         f"{what} out vs oracle on the GPU's set")
+    else:
+        assert_out_close(gpu_out, np.zeros_like(np.asarray(gpu_out, dtype=np.float64)),
+                         f"{what} empty selection")
+    # the oracle's own step output, where its selection is the GPU's (with tau
+    # calibrated on the same scores, t sits on a score, and one entry more or
+    # less -- inside the band -- moves the output by its whole weight)
+    out_ref, idx_ref, _ = oracle.step_row(np.asarray(q_row), np.asarray(k_rows),
+                                          np.asarray(v_rows), tau, TAIL, cap)
+    if np.array_equal(idx_ref, sel):
+        assert_out_close(gpu_out, out_ref, f"{what} out vs oracle step")
+    return n

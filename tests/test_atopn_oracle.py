@@ -85,3 +85,13 @@ def test_step_with_everything_selected_is_dense_attention():
     # the exact oracle with N = L is the same dense attention
     ref = oracle.combine(z, v)
     np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_threshold_above_every_probability_selects_nothing():
+    # the row's largest probability is 1/2 (z = [0, 0, ln 2]); tau = 0.6 is above it
+    z = np.array([0.0, 0.0, math.log(2.0)])
+    assert ao.step_select(z, 0.6, 1, cap=6).size == 0
+    k = np.eye(3, 4) * 2.0
+    q = np.array([0.0, 0.0, math.log(2.0), 0.0])
+    out, idx, _ = ao.step_row(q, k, np.ones((3, 4)), 0.9, 1, cap=6)
+    assert idx.size == 0 and np.all(out == 0.0)
