@@ -371,6 +371,50 @@ def run_saga(args, rank, world, local):
     e2e_ms = max_over_ranks(h0.elapsed_time(h1), world)
     if not torch.equal(pin_o[0], outs[0].cpu()):
         raise RuntimeError("host entry point result differs from the device call")
+
+    # ---- stateful Atop-N: tau calibrated once per layer, then the step call (the
+    # calibrated threshold reused, "More Value per Key" App. C.1), graphed and timed
+    # like the headline on the same caches and queries
+    taus = []
+    for x, o in zip(layers, outs):
+        taus.append(dec.atopn_calibrate(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=o)[1])
+
+    def step_atopn():
+        for x, o, lt in zip(layers, outs, taus):
+            dec.atopn_step(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, lt, out=o)
+
+    step_atopn()
+    a_status = dec.status()
+    if a_status & 0xFF:
+        raise RuntimeError(f"device status 0x{a_status:x} in the Atop-N step")
+    a_sel = torch.empty(B, spec.h_q, 2 * spec.N, dtype=torch.int32, device=dev)
+    dec.atopn_step(x0.q, x0.k_cache, x0.v_cache, x0.seq_lens, spec.N, taus[0], out=outs[0],
+                   sel_idx=a_sel,
+                   sel_logit=torch.empty(B, spec.h_q, 2 * spec.N, dtype=torch.float32, device=dev))
+    a_kept = (a_sel >= 0).sum(-1).float()
+    with torch.cuda.stream(side):
+        step_atopn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    n1 = dec.launch_count()
+    agraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(agraph):
+        step_atopn()
+    a_launches = dec.launch_count() - n1
+    for _ in range(max(args.warmup, 3)):
+        agraph.replay()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(args.steps):
+        agraph.replay()
+    a1.record()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    a_ms = max_over_ranks(a0.elapsed_time(a1), world)
+    a_status = dec.status()
     if clocks:
         clocks.stop()
 
@@ -447,6 +491,16 @@ def run_saga(args, rank, world, local):
         },
         "gpu_launches": launches_per_step * args.steps,
         "clocks": csum,
+        "atopn_step": {
+            "what": "stateful Atop-N step (saga_atopn_step): tau calibrated once per layer on "
+                    "the same caches and queries, so the threshold is the N-th score up to "
+                    "rounding; 2N-entry buffer",
+            "value": world * B / (a_ms / 1e3 / args.steps) * L / spec.layers,
+            "unit": "tokens/s", "ms_per_step": a_ms / args.steps,
+            "gpu_launches": a_launches * args.steps,
+            "kept_per_row_mean": float(a_kept.mean()), "kept_per_row_max": int(a_kept.max()),
+            "robust_path_seen": bool(a_status & 0x200),
+        },
     }
     print(json.dumps(line), flush=True)
 

@@ -23,11 +23,11 @@
 //     scale, and either store z row-wise (coalesced per head) with per-(b, j)
 //     min/max statistics, or append the candidates of the selector.
 //
-// With kLse (candidate mode), the epilogue also writes, per query head
-// and 32-position chunk, the sum of exp(z - m_ref[row]) over the chunk's
-// positions: the pieces of the row's log-sum-exp, from which a calibrated
+// With kLse (candidate mode), the epilogue also writes, per query head and
+// 32-position chunk slot, sums of exp(z - m_ref[row]) that add up over a row to
+// the row's total: the pieces of its log-sum-exp, from which a calibrated
 // probability threshold becomes a logit threshold ("More Value per Key",
-// App. C.1).  A term whose exponent exceeds kLseMaxExp makes the chunk's sum
+// App. C.1).  A term whose exponent exceeds kLseMaxExp makes the row's sum
 // +inf, which sends the row to the selector's exact fallback.
 #pragma once
 
@@ -51,7 +51,7 @@ struct ScoreParams {
   long long mask_stride;
   const float* t_lo;         // [B*h_q] candidate bounds, written by the preceding kernel
   const float* m_ref;        // [B*h_q] exp-sum references (+inf: no sums), with lse_part
-  float* lse_part;           // [B*h_q][mask_stride] per-chunk sums of exp(z - m_ref) (kLse)
+  float* lse_part;           // [B*h_q][mask_stride] chunk slots of the sums of exp(z - m_ref) (kLse)
   uint32_t* stat_min;        // [B*h_q] ordered keys, or nullptr
   uint32_t* stat_max;
   int* status;
@@ -369,6 +369,27 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int e = 0; e < H; ++e) { tl[e] = INFINITY; mr[e] = INFINITY; }
     static_assert(kCand || !kLse, "chunk sums come with the candidate mode");
     constexpr bool lse = kLse;
+    // kLse: this lane's running sums of exp(z - m_ref) over the warp's tiles of
+    // the current row segment (its "piece"); when the piece ends, one butterfly
+    // gives the per-head totals, which go to the slot of the piece's first
+    // chunk; every other chunk of the piece gets 0 (so a row's slots still add
+    // up to its sum, in a fixed order).
+    float ls[H];
+    int ls_chunk = -1, ls_row0 = 0;
+#pragma unroll
+    for (int e = 0; e < H; ++e) ls[e] = 0.0f;
+    auto flush_lse = [&]() {
+      if (!lse || ls_chunk < 0) return;          // uniform
+      constexpr int kSpread = H <= 16 ? 2 : 1;   // lanes per head in the result
+      const float sum = warp_transpose_sum<H>(ls, lane);
+      const int e = lane / kSpread;
+      if (lane % kSpread == 0 && e < H && h0 + e < p.g)
+        st_global_hint(p.lse_part + static_cast<long long>(ls_row0 + e) * p.mask_stride + ls_chunk,
+                       sum, pol_z);
+#pragma unroll
+      for (int e2 = 0; e2 < H; ++e2) ls[e2] = 0.0f;
+      ls_chunk = -1;
+    };
     if (n_tiles > 0) {
       TileCursor c;
       c.seek(u0, unit_off, lens, p.B, p.h_k);
@@ -377,6 +398,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (!alive || i % TG != tg) continue;
         if (c.b != seg_b || c.kh != seg_kh) {     // a new row segment
           if (!kCand) flush();
+          flush_lse();
           seg_b = c.b;
           seg_kh = c.kh;
           if (kCand) {
@@ -399,14 +421,13 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int chunk = c.t * (kTileM / 32) + quad;
           uint32_t* kslot = reinterpret_cast<uint32_t*>(p.z) + static_cast<long long>(row0) * p.z_stride + chunk * 32;
           uint32_t my_m = 0u;
-          float ex[H];
 #pragma unroll
           for (int e = 0; e < H; ++e) {
             // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
             const float zz = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
             if (lse) {   // exp(-inf) = 0 for rows without a reference
               const float a = zz - mr[e];
-              ex[e] = (valid && h0 + e < p.g) ? (a > kLseMaxExp ? INFINITY : expf(a)) : 0.0f;
+              ls[e] += (valid && h0 + e < p.g) ? (a > kLseMaxExp ? INFINITY : __expf(a)) : 0.0f;
             }
             const bool take = valid && h0 + e < p.g && zz >= tl[e];
             const uint32_t m = __ballot_sync(0xffffffffu, take);
@@ -417,12 +438,14 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           if (lane < H && h0 + lane < p.g && chunk * 32 < c.Lb)   // lane e: head e's mask
             st_global_hint(p.cand_mask + static_cast<long long>(row0 + lane) * p.mask_stride + chunk, my_m, pol_z);
-          if (lse) {
-            constexpr int kSpread = H <= 16 ? 2 : 1;             // lanes per head in the result
-            const float sum = warp_transpose_sum<H>(ex, lane);
-            const int e = lane / kSpread;
-            if (lane % kSpread == 0 && e < H && h0 + e < p.g && chunk * 32 < c.Lb)
-              st_global_hint(p.lse_part + static_cast<long long>(row0 + e) * p.mask_stride + chunk, sum, pol_z);
+          if (lse && chunk * 32 < c.Lb) {
+            if (ls_chunk < 0) {                  // the piece's first chunk takes its total
+              ls_chunk = chunk;
+              ls_row0 = row0;
+            } else if (lane < H && h0 + lane < p.g) {
+              st_global_hint(p.lse_part + static_cast<long long>(row0 + lane) * p.mask_stride + chunk,
+                             0.0f, pol_z);
+            }
           }
         } else if (valid) {
           float* zrow = p.z + static_cast<long long>(row0) * p.z_stride + pos;
@@ -440,6 +463,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
       if (!kCand) flush();
+      flush_lse();
     }
   }
 

@@ -92,15 +92,19 @@ EPS32 = 2.0 ** -24
 def lse_error(q_row, k_rows, z_ref, extra=0.0):
     """The row's float64 log-sum-exp and a bound on the error of the GPU's fp32 one.
 
-    The GPU sums exp(z) of its fp32 scores: d(LSE)/dz_i = p_i, so the scores'
-    errors move it by at most sum_i p_i * bound_i; the sum itself (exp within
-    2 ulp, a reduction tree of depth < 32) adds 32 ulp relative, and the fp32
-    values of magnitude |LSE| and |extra| combined with it a few ulp each."""
+    The GPU sums exp(z - m_ref) of its fp32 scores, m_ref one of the row's
+    sampled scores: d(LSE)/dz_i = p_i, so the scores' errors move it by at most
+    sum_i p_i * bound_i; the fast exp is within 2 + 1.17 |x| ulp for an
+    argument x (|x| <= the row's score range), the sums add at most 32 ulp
+    relative (reduction depth < 32), and the fp32 values of magnitude |LSE| and
+    |extra| combined with it a few ulp each."""
     m = z_ref.max()
     e = np.exp(z_ref - m)
     lse = m + math.log(e.sum())
     p = e / e.sum()
-    err = float(p @ score_bound(q_row, k_rows)) + 32 * EPS32 + 8 * EPS32 * (abs(lse) + abs(extra))
+    spread = float(z_ref.max() - z_ref.min())
+    err = (float(p @ score_bound(q_row, k_rows)) + (34 + 1.17 * spread) * EPS32 +
+           8 * EPS32 * (abs(lse) + abs(extra)))
     return lse, err
 
 
