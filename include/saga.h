@@ -95,7 +95,7 @@ typedef struct saga_ctx* saga_handle;
  * head_dim, and selections of up to max_N positions.  cuda_stream is a
  * cudaStream_t (NULL = legacy default stream).  The current CUDA device at
  * this call is the handle's device.  Workspace: about
- * 4*max_batch*h_q*(round_up(max_seq_len,32)*17/16 + 4*max_N + 1030 +
+ * 4*max_batch*h_q*(round_up(max_seq_len,32)*17/16 + 4*max_N + 1029 + head_dim +
  * ceil(min(max_N,max_seq_len)/256)*(head_dim+2)) bytes.
  * Returns SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_CUDA. */
 SAGA_API int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len,
