@@ -7,8 +7,10 @@ from .saga_oracle import (head_maps, scores, top_n, nth_score, softmax_selected,
                           gathered_pv, decode_row, decode_attn, combine)
 from .atopn_oracle import (calibrate_tau, tail_max, step_threshold, step_select,
                            step_row, calibrate_row, step_attn)
+from .group_oracle import group_statistic, group_select, group_rows, group_attn
 
 __all__ = ["head_maps", "scores", "top_n", "nth_score", "softmax_selected",
            "gathered_pv", "decode_row", "decode_attn", "combine",
            "calibrate_tau", "tail_max", "step_threshold", "step_select",
-           "step_row", "calibrate_row", "step_attn"]
+           "step_row", "calibrate_row", "step_attn",
+           "group_statistic", "group_select", "group_rows", "group_attn"]
