@@ -37,6 +37,17 @@
 // Both set INFO_ROBUST_PATH in the status word.  Keys are order-preserving
 // uint32 images of the fp32 scores, -0 folded onto +0; ties at the N-th score
 // go to the lowest position.  NaN scores are not supported.
+//
+// Stateful Atop-N (App. C.1) adds two modes.  Both need the row's log-sum-exp:
+// from the score pass's chunk sums of exp(z - m_ref), read in the same round
+// as the masks (rows longer than the candidate cap), else from the complete
+// candidate list.  Calibration runs steps 1-5 and writes log tau = z(T) -
+// logsumexp.  A step replaces 3 and 4 by t = log tau + logsumexp and one
+// ordered pass that keeps every key >= key(t), the first 2N in position order
+// (one block scan per pass), then takes the softmax weights over the kept
+// logits.  The step's candidates cover t whenever t >= t_lo (the bound is for
+// the 2N-th score); otherwise, or when the chunk sums left the fp32 range, the
+// row is scored again here and its log-sum-exp taken from those keys.
 #pragma once
 
 #include <cuda_bf16.h>
