@@ -110,6 +110,34 @@ def test_full_size_sampled_rows(spec):
     assert torch.isfinite(out.float()).all()
 
 
+SWEEP = {s.name: s for s in workload.sweep_specs()}
+SWEEP_POINTS = ["qwen_sweep_b1_l128k_n2048", "qwen_sweep_b8_l32k_n1024",
+                "qwen_sweep_b64_l8k_n512", "qwen_sweep_b64_l128k_n512"]
+
+
+@pytest.mark.parametrize("name", SWEEP_POINTS)
+def test_sweep_points_sampled_rows(name):
+    # Corners of the long-context sweep (Qwen shapes, 1% planted keys), inputs drawn
+    # on the device; rows of 128K positions take the slot path (INFO_ROBUST_PATH).
+    spec = SWEEP[name]
+    inp = workload.make_inputs(spec, device="cuda")
+    dec = SagaDecoder(spec.batch, spec.seq_len, spec.h_q, spec.h_k, spec.h_v, spec.head_dim, spec.N)
+    out, idx, logit, st = run_decode(dec, inp.q, inp.k_cache, inp.v_cache, inp.seq_lens, spec.N)
+    assert st & 0xFF == 0
+    rng = np.random.default_rng(len(name))
+    rows = {(int(rng.integers(spec.batch)), int(rng.integers(spec.h_q))) for _ in range(3)}
+    rows |= {(0, 0), (spec.batch - 1, spec.h_q - 1)}
+    check_rows(inp, spec.h_q, spec.h_k, spec.h_v, spec.N, out, idx, logit, sorted(rows))
+    idx_c = idx.cpu()
+    assert (idx_c[..., 1:] > idx_c[..., :-1]).all() and (idx_c[..., 0] >= 0).all()
+    keep = {}
+    for b, j, pos in inp.planted:
+        keep.setdefault((b, j), []).append(pos)
+    for (b, j), pos in keep.items():
+        assert set(pos) <= set(idx_c[b, j].tolist()), f"planted keys of ({b}, {j}) not selected"
+    assert torch.isfinite(out.float()).all()
+
+
 # --------------------------------------------------------------------------- shapes and edges
 
 SHAPES = [
