@@ -207,6 +207,22 @@ def oracle_sample(spec, q, k, v, lens, budget_s):
     return rows, spent, threads
 
 
+def cpp_oracle_sample(spec, q, k, v, lens):
+    """Time the plain C++ oracle on batch row 0 of one layer (all heads), on one
+    thread and on every core; returns (single-thread s, all-core s, cores)."""
+    import numpy as np
+    from oracle import cref
+    cores = os.cpu_count() or 1
+    qb, kb, vb = q[0:1].cpu(), k[0:1].cpu(), v[0:1].cpu()
+    lb = np.array([int(lens[0])], dtype=np.int32)
+    times = []
+    for threads in (1, cores):
+        t0 = time.perf_counter()
+        cref.decode(qb, kb, vb, lb, spec.h_q, spec.h_k, spec.h_v, spec.N, threads=threads)
+        times.append(time.perf_counter() - t0)
+    return times[0], times[1], cores
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: each step is one batch row of one layer."""
     from sparse_asymmetric_gqa_b200 import workload
@@ -438,6 +454,8 @@ def run_saga(args, rank, world, local):
     rows, spent, threads = oracle_sample(spec, layers[0].q, layers[0].k_cache, layers[0].v_cache,
                                          lens, args.cpu_seconds)
     cpu_tok_s = rows / (spent * spec.layers)
+    cpp_1, cpp_all, cpp_cores = cpp_oracle_sample(spec, layers[0].q, layers[0].k_cache,
+                                                  layers[0].v_cache, lens)
     csum = clocks.summary(t_wall0, t_wall1) if clocks else {}
     line = {
         "metric": METRIC,
@@ -481,6 +499,12 @@ def run_saga(args, rank, world, local):
             "value": cpu_tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{rows} batch rows x 12 heads of layer 0 ({spent:.1f} s of CPU work), "
                       "scaled by 28 layers per token",
+        },
+        "cpu_oracle_cpp": {
+            "kind": "plain C++ oracle (double, std::thread over rows)",
+            "single_thread_tokens_per_s": 1.0 / (cpp_1 * spec.layers),
+            "all_cores_tokens_per_s": 1.0 / (cpp_all * spec.layers), "cores": cpp_cores,
+            "sample": "batch row 0 x 12 heads of layer 0, scaled by 28 layers per token",
         },
         "e2e": {
             "value": world * B / e2e_step_s, "unit": "tokens/s",
