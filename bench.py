@@ -207,6 +207,17 @@ def oracle_sample(spec, q, k, v, lens, budget_s):
     return rows, spent, threads
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpp_oracle_sample(spec, q, k, v, lens):
     """Time the plain C++ oracle on batch row 0 of one layer (all heads), on one
     thread and on every core; returns (single-thread s, all-core s, cores)."""
@@ -504,6 +515,7 @@ def run_saga(args, rank, world, local):
             "kind": "plain C++ oracle (double, std::thread over rows)",
             "single_thread_tokens_per_s": 1.0 / (cpp_1 * spec.layers),
             "all_cores_tokens_per_s": 1.0 / (cpp_all * spec.layers), "cores": cpp_cores,
+            "cpu_model": cpu_model(),
             "sample": "batch row 0 x 12 heads of layer 0, scaled by 28 layers per token",
         },
         "e2e": {
