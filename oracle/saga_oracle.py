@@ -9,8 +9,10 @@ What it computes is the plain definition, in float64, written from
 "More Value per Key: Asymmetric Sparse Attention for Faster LLM Decoding"
 (Elata et al.), cited below as [MVK]:
 
-* scores      z_i = q . k_i / sqrt(d) over every cached position, the current
-                token included                      [MVK] §2.1 Eq. (2), §2.2 Eq. (5)
+* scores      z_i = q . k_i / sqrt(d_k) over every cached position, the current
+                token included (d_k the query/key width; values may be wider,
+                d_v, as in the pages' key-dimension variant, [MVK] §5.2)
+                                                    [MVK] §2.1 Eq. (2), §2.2 Eq. (5)
 * selection   i = TopN(z): the N largest entries of the score row of each query
               head; everything else is masked       [MVK] §2.5 Eq. (6)
 * softmax     over the gathered (selected) logits only; padding slots get zero
@@ -35,7 +37,8 @@ Readings where the pages are silent (each also listed in the design notes):
 
 Parity pins: every function here is pinned in ``tests/test_oracle_pins.py``
 against closed forms, a pure-Python brute force, torch's float64
-``scaled_dot_product_attention`` and structural invariants.  No function is
+``scaled_dot_product_attention`` and structural invariants (and, for keys
+narrower than values, in ``tests/test_oracle_dkdv.py``).  No function is
 "parity unpinned".
 
 Inputs are numpy arrays whose values are exactly representable in bf16 (the
@@ -112,9 +115,9 @@ def decode_row(q, k_cache, v_cache, seq_lens, b: int, j: int,
                h_q: int, h_k: int, h_v: int, N: int):
     """One (batch row, query head) of the decode step.
 
-    q: [B, h_q, d]; k_cache: [B, h_k, L_max, d]; v_cache: [B, h_v, L_max, d];
+    q: [B, h_q, d_k]; k_cache: [B, h_k, L_max, d_k]; v_cache: [B, h_v, L_max, d_v];
     seq_lens: [B] (positions 0..L_b-1 are valid, the current token at L_b-1).
-    Returns (out [d] float64, idx [N_b] ascending, z_sel [N_b], z [L_b]).
+    Returns (out [d_v] float64, idx [N_b] ascending, z_sel [N_b], z [L_b]).
     """
     key_head, value_head = head_maps(h_q, h_k, h_v)
     L_b = int(seq_lens[b])
@@ -129,11 +132,11 @@ def decode_row(q, k_cache, v_cache, seq_lens, b: int, j: int,
 def decode_attn(q, k_cache, v_cache, seq_lens, h_q: int, h_k: int, h_v: int, N: int):
     """The whole decode step for every (b, j).
 
-    Returns (out [B, h_q, d] float64, idx list-of-lists, z_sel list-of-lists).
+    Returns (out [B, h_q, d_v] float64, idx list-of-lists, z_sel list-of-lists).
     """
     B = q.shape[0]
-    d = q.shape[-1]
-    out = np.zeros((B, h_q, d), dtype=np.float64)
+    d_v = v_cache.shape[-1]          # the output has the value width (d_v may differ from d_k)
+    out = np.zeros((B, h_q, d_v), dtype=np.float64)
     idx_all, zsel_all = [], []
     for b in range(B):
         idx_b, zsel_b = [], []
