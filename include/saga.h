@@ -221,6 +221,13 @@ SAGA_API int saga_combine_noalloc(const int32_t* sel_idx, const float* sel_logit
  * set, else SAGA_OK. */
 SAGA_API int saga_decode_status(saga_handle h, int* device_status);
 
+/* Failure-detection self-test: enqueues one kernel whose bounded pipeline wait
+ * has nothing to wait for.  After the wait's limit (2 s) the kernel sets
+ * SAGA_STATUS_TIMEOUT in the device status word and exits, as a stalled
+ * pipeline stage would; saga_decode_status then returns SAGA_ERR_DEVICE with
+ * that bit, and the handle and the CUDA context stay usable.  Asynchronous. */
+SAGA_API int saga_decode_selftest_timeout(saga_handle h);
+
 /* Total number of kernels this handle has launched. */
 SAGA_API int saga_decode_launch_count(saga_handle h, long long* count);
 

@@ -226,6 +226,12 @@ class SagaDecoder:
             raise SagaError("saga_decode_status", rc)
         return v.value
 
+    def selftest_timeout(self):
+        """Failure-detection self-test: a kernel whose bounded wait runs out sets
+        SAGA_STATUS_TIMEOUT (read it with ``status()``); asynchronous, ~2 s."""
+        self._stream()
+        _lib.check("saga_decode_selftest_timeout", self.lib.saga_decode_selftest_timeout(self._h))
+
     def launch_count(self) -> int:
         v = ctypes.c_longlong(0)
         _lib.check("saga_decode_launch_count", self.lib.saga_decode_launch_count(self._h, ctypes.byref(v)))

@@ -349,6 +349,20 @@ int launch_gather(saga_ctx* h, const int32_t* sel_idx, const float* sel_logit,
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
+// Failure-detection self-test: one thread waits, with the pipeline's bounded
+// wait, on an mbarrier that nothing arrives at; when the wait gives up it sets
+// SAGA_STATUS_TIMEOUT, as a stalled pipeline stage would.
+__global__ void selftest_wait_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_addr(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    volatile int never = 0;
+    if (!mbar_wait(b, 0, &never)) atomicOr(status, 0x2 /* SAGA_STATUS_TIMEOUT */);
+  }
+}
+
 int check_heads(saga_ctx* h, int h_q, int h_k, int h_v, int d) {
   if (h_q != h->h_q || h_k != h->h_k || h_v != h->h_v || d != h->d) return SAGA_ERR_INVALID_ARG;
   return SAGA_OK;
@@ -576,6 +590,14 @@ int saga_atopn_step(saga_handle h, const void* q, const void* k_cache, const voi
   if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
   return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit, kModeStep,
                      const_cast<float*>(log_tau));
+}
+
+int saga_decode_selftest_timeout(saga_handle h) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  return launch(h, selftest_wait_kernel, dim3(1), dim3(32), 0, kPlain, h->status) == cudaSuccess
+             ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache,

@@ -356,3 +356,19 @@ def test_batch_smaller_than_max():
     assert st == 0
     check_rows(inp, spec.h_q, spec.h_k, spec.h_v, spec.N, out, idx, logit,
                [(b, j) for b in range(4) for j in range(0, spec.h_q, 3)])
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    # Failure detection without a fault: a pipeline wait with nothing to wait for
+    # gives up after its limit, the status word says SAGA_STATUS_TIMEOUT, and the
+    # handle keeps working (the next decode call is clean and correct).
+    spec = workload.TINY
+    inp = workload.make_inputs(spec)
+    dec = SagaDecoder(spec.batch, spec.seq_len, spec.h_q, spec.h_k, spec.h_v, spec.head_dim, spec.N)
+    dec.selftest_timeout()
+    st = dec.status()
+    assert st & _lib.SAGA_STATUS_TIMEOUT
+    out, idx, logit, st = run_decode(dec, *_dev(inp), spec.N)
+    assert st == 0
+    check_rows(inp, spec.h_q, spec.h_k, spec.h_v, spec.N, out, idx, logit,
+               [(0, j) for j in range(spec.h_q)])
