@@ -359,6 +359,18 @@ def run_saga(args, rank, world, local):
     ms = e0.elapsed_time(e1)
     ms_max = max_over_ranks(ms, world)
 
+    # per-replay times in a separate pass (an event after every replay), for the median
+    n_med = max(1, min(args.steps, 50))
+    rev = [torch.cuda.Event(enable_timing=True) for _ in range(n_med + 1)]
+    rev[0].record()
+    for r in range(n_med):
+        graph.replay()
+        rev[r + 1].record()
+    torch.cuda.synchronize(dev)
+    per_replay = sorted(rev[r].elapsed_time(rev[r + 1]) for r in range(n_med))
+    median_ms = max_over_ranks(per_replay[n_med // 2] if n_med % 2 else
+                               0.5 * (per_replay[n_med // 2 - 1] + per_replay[n_med // 2]), world)
+
     # ---- per-kernel times: the profiled graph, same number of steps
     for _ in range(max(args.warmup, 3)):
         pgraph.replay()
@@ -476,6 +488,7 @@ def run_saga(args, rank, world, local):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps,
+        "ms_per_step_median": median_ms,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
