@@ -209,7 +209,10 @@ SAGA_API int saga_combine(saga_handle h, const int32_t* sel_idx, const float* se
  * device looks up the array's device address; make that first call before any stream
  * capture.  Every call clears the part of the array that must start at zero and reuses the
  * rest, so calls that can overlap on the GPU (different streams) race and must not be issued
- * concurrently.  Rows with seq_lens[b] outside [1, max_seq_len] get zeros.  Asynchronous. */
+ * concurrently.  Device-side data errors are handled as in saga_combine but not reported:
+ * with no handle there is no status word to read, so a row with seq_lens[b] outside
+ * [1, max_seq_len] gets zeros and an entry with an index >= seq_lens[b] is skipped, silently
+ * (a caller that needs the report uses saga_combine).  Asynchronous. */
 SAGA_API int saga_combine_noalloc(const int32_t* sel_idx, const float* sel_logit,
                                   const void* v_cache, const int32_t* seq_lens, int batch,
                                   int max_seq_len, int h_q, int h_v, int head_dim, int N,

@@ -270,7 +270,10 @@ def combine_noalloc(sel_idx, sel_logit, v_cache, seq_lens, out):
     SagaError (SAGA_ERR_SCRATCH_TOO_SMALL).  The first call on a device should come before
     any stream capture, and calls on different streams must not overlap on the GPU.
     sel_idx / sel_logit: [B, h_q, N] (index -1 = padding); v_cache: [B, h_v, L_max, d] bf16;
-    seq_lens: [B] int32.  Runs on the current stream, asynchronously.
+    seq_lens: [B] int32, all on out's device.  Runs on that device's current stream,
+    asynchronously.  Data errors only the device sees are not reported (there is no handle
+    and so no status word): a row whose seq_len lies outside [1, L_max] gets zeros and an
+    index >= its row's seq_len is skipped.
     """
     lib = load()
     B, h_q, N = sel_idx.shape
@@ -282,8 +285,14 @@ def combine_noalloc(sel_idx, sel_logit, v_cache, seq_lens, out):
     _, h_v, L_max, d = v_cache.shape
     _need(seq_lens, "seq_lens", torch.int32, (B,), "cuda")
     _need(out, "out", torch.bfloat16, (B, h_q, d), "cuda")
-    stream = torch.cuda.current_stream(out.device).cuda_stream
-    _lib.check("saga_combine_noalloc", lib.saga_combine_noalloc(
-        _ptr(sel_idx), _ptr(sel_logit), _ptr(v_cache), _ptr(seq_lens), B, L_max, h_q, h_v, d, N,
-        _ptr(out), ctypes.c_void_p(stream)))
+    for name, t in (("sel_idx", sel_idx), ("sel_logit", sel_logit), ("v_cache", v_cache),
+                    ("seq_lens", seq_lens)):
+        if t.device != out.device:
+            raise ValueError(f"{name} is on {t.device}, out on {out.device}: one device for all")
+    # the library looks up its scratch on the current device and runs on its current stream
+    with torch.cuda.device(out.device):
+        stream = torch.cuda.current_stream(out.device).cuda_stream
+        _lib.check("saga_combine_noalloc", lib.saga_combine_noalloc(
+            _ptr(sel_idx), _ptr(sel_logit), _ptr(v_cache), _ptr(seq_lens), B, L_max, h_q, h_v, d,
+            N, _ptr(out), ctypes.c_void_p(stream)))
     return out
