@@ -224,6 +224,26 @@ SAGA_API int saga_combine_noalloc(const int32_t* sel_idx, const float* sel_logit
  * set, else SAGA_OK. */
 SAGA_API int saga_decode_status(saga_handle h, int* device_status);
 
+/* Group-shared selection (a different method from the decode step: results
+ * differ): the g_v = h_q/h_v query heads that read one value head share one set
+ * of N positions -- the N_b largest s_i = sum over the group's heads j of
+ * softmax(z_j)_i (the GQA form of SparQ's position step as the pages describe
+ * it, applied to [MVK] §3.1 Eq. (7), §3.2), ties to the lowest position -- and
+ * each head takes the softmax of its own logits over the set and the gathered
+ * P.V, so the value gather reads N rows per value head.
+ *   sel_idx   int32 [B][h_v][N]   the shared positions, ascending, -1 padding
+ *   sel_stat  fp32  [B][h_v][N]   s at them, -inf padding
+ *   sel_logit fp32  [B][h_q][N]   each head's logits at them, -inf padding
+ * (each may be NULL).  Needs h_k | h_v, g = h_q/h_k <= 32, g_v <= 8,
+ * N <= min(max_N, 1024) and N * g_v <= 8192, else SAGA_ERR_UNSUPPORTED.  Rows
+ * whose kept positions cannot be shown to contain the top N of s are scored
+ * again on CUDA cores (SAGA_STATUS_INFO_ROBUST_PATH).  Layouts, ownership and
+ * errors as saga_decode_attn_ex. */
+SAGA_API int saga_group_attn(saga_handle h, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* seq_lens, int h_q, int h_k,
+                             int h_v, int head_dim, int N, void* out, int32_t* sel_idx,
+                             float* sel_stat, float* sel_logit);
+
 /* Failure-detection self-test: enqueues one kernel whose bounded pipeline wait
  * has nothing to wait for.  After the wait's limit (2 s) the kernel sets
  * SAGA_STATUS_TIMEOUT in the device status word and exits, as a stalled

@@ -106,6 +106,28 @@ class SagaDecoder:
                        self.lib.saga_decode_attn_ex(*args, _ptr(sel_idx), _ptr(sel_logit)))
         return out
 
+    def group_attn(self, q, k_cache, v_cache, seq_lens, N: int, out=None, sel_idx=None,
+                   sel_stat=None, sel_logit=None):
+        """Group-shared selection: one set of N positions per value head (the largest
+        summed softmax probabilities of its query heads), each head's own softmax over
+        it and the gathered P.V.  sel_idx / sel_stat [B, h_v, N], sel_logit [B, h_q, N]."""
+        self._check_caches(q, k_cache, v_cache, seq_lens)
+        B = self.batch
+        if out is None:
+            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+        if sel_idx is not None:
+            _need(sel_idx, "sel_idx", torch.int32, (B, self.h_v, N), "cuda")
+        if sel_stat is not None:
+            _need(sel_stat, "sel_stat", torch.float32, (B, self.h_v, N), "cuda")
+        if sel_logit is not None:
+            _need(sel_logit, "sel_logit", torch.float32, (B, self.h_q, N), "cuda")
+        self._stream()
+        _lib.check("saga_group_attn", self.lib.saga_group_attn(
+            self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), self.h_q, self.h_k,
+            self.h_v, self.head_dim, N, _ptr(out), _ptr(sel_idx), _ptr(sel_stat), _ptr(sel_logit)))
+        return out
+
     def atopn_calibrate(self, q, k_cache, v_cache, seq_lens, N: int, log_tau=None, out=None,
                         sel_idx=None, sel_logit=None):
         """Calibration step of stateful Atop-N: the exact top-N decode step, and per row

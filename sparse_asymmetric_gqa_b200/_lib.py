@@ -36,6 +36,7 @@ SIGNATURES = {
     "saga_combine_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "saga_decode_status": (_I, [_P, ctypes.POINTER(_I)]),
     "saga_decode_selftest_timeout": (_I, [_P]),
+    "saga_group_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "saga_decode_launch_count": (_I, [_P, ctypes.POINTER(ctypes.c_longlong)]),
     "saga_decode_profile": (_I, [_P, _I, _I]),
     "saga_decode_profile_read": (_I, [_P, ctypes.POINTER(ctypes.c_double),

@@ -9,7 +9,8 @@ LIB = os.path.join(HERE, "libsaga.so")
 SOURCES = [os.path.join(HERE, "csrc", "saga_api.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "score_kernel.cuh",
                                                           "select_kernel.cuh", "gather_kernel.cuh",
-                                                          "topn_kernel.cuh", "bound_kernel.cuh")] + \
+                                                          "topn_kernel.cuh", "bound_kernel.cuh",
+                                                          "group_kernel.cuh")] + \
     [os.path.join(ROOT, "include", "saga.h")]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",

@@ -34,6 +34,7 @@
 #include "gather_kernel.cuh"
 #include "topn_kernel.cuh"
 #include "bound_kernel.cuh"
+#include "group_kernel.cuh"
 
 using namespace saga;
 
@@ -101,6 +102,8 @@ struct saga_ctx {
   float* t_lo = nullptr;          // candidate bounds [rows]
   float* m_ref = nullptr;         // exp-sum references [rows] (calibration and steps)
   float* lse_part = nullptr;      // chunk sums of exp(z - m_ref) [rows][mask_stride]
+  uint32_t* gstat = nullptr;      // group statistic keys [max_batch * h_v][z_stride]
+  float* gsel_stat = nullptr;     // group statistic at the selection [max_batch * h_v][max_N]
   float* partial = nullptr;       // gather partials [rows][max_chunks][d + 2]
   uint32_t* counter = nullptr;    // gather merge counters [rows]
   int max_chunks = 0;
@@ -131,9 +134,21 @@ int set_smem_attrs_once() {
     SAGA_ATTR(64, 16) SAGA_ATTR(64, 32) SAGA_ATTR(64, 48) SAGA_ATTR(64, 64)
     SAGA_ATTR(128, 16) SAGA_ATTR(128, 32) SAGA_ATTR(128, 48) SAGA_ATTR(128, 64)
 #undef SAGA_ATTR
+#define SAGA_GATTR(D, NP)                                                                         \
+  if (e == cudaSuccess)                                                                           \
+    e = cudaFuncSetAttribute(score_kernel<D, NP, true, true, true>,                               \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes);
+    SAGA_GATTR(64, 16) SAGA_GATTR(64, 32) SAGA_GATTR(128, 16) SAGA_GATTR(128, 32)
+#undef SAGA_GATTR
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sizeof(SelectSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(group_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(group_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
 #define SAGA_TOPN_ATTR(D, M, S)                                                                   \
   if (e == cudaSuccess)                                                                           \
     e = cudaFuncSetAttribute(topn_kernel<D, M, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
@@ -181,7 +196,8 @@ cudaError_t launch(saga_ctx* h, void (*kernel)(KArgs...), dim3 grid, dim3 block,
 // candidate keys in the workspace; a programmatic dependent of the bound
 // kernel); otherwise every score goes to z.
 int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t* seq_lens,
-                 float* z, long long z_stride, bool stats, bool cand = false, bool lse = false) {
+                 float* z, long long z_stride, bool stats, bool cand = false, bool lse = false,
+                 bool group = false) {
   CUtensorMap mk, mq;
   const uint64_t k_rows = static_cast<uint64_t>(h->batch) * h->h_k * h->max_seq_len;
   const uint64_t q_rows = static_cast<uint64_t>(h->batch) * h->h_q;
@@ -210,14 +226,23 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
       static_cast<long long>(h->batch) * h->h_k * ((h->max_seq_len + kTileM - 1) / kTileM);
   const int grid = static_cast<int>(max_units < h->num_sms ? max_units : h->num_sms);
   cudaError_t e = cudaErrorInvalidValue;
+  if (group) {   // group candidates (g <= 32)
+#define SAGA_GCASE(D, NP)                                                                      \
+    if (h->d == D && h->npad == NP)                                                            \
+      e = launch(h, score_kernel<D, NP, true, true, true>, dim3(grid), dim3(kScoreThreads),    \
+                 ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p, h->g_v);
+    SAGA_GCASE(64, 16) SAGA_GCASE(64, 32) SAGA_GCASE(128, 16) SAGA_GCASE(128, 32)
+#undef SAGA_GCASE
+    return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
+  }
 #define SAGA_CASE(D, NP)                                                                       \
   if (h->d == D && h->npad == NP)                                                              \
     e = (cand && lse) ? launch(h, score_kernel<D, NP, true, true>, dim3(grid), dim3(kScoreThreads), \
-                               ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p)                  \
+                               ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p, h->g_v)                  \
       : cand ? launch(h, score_kernel<D, NP, true>, dim3(grid), dim3(kScoreThreads),           \
-                      ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p)                          \
+                      ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p, h->g_v)                          \
              : launch(h, score_kernel<D, NP, false>, dim3(grid), dim3(kScoreThreads),          \
-                      ScoreShape<D, NP>::kSmemBytes, kPlain, mk, mq, p);
+                      ScoreShape<D, NP>::kSmemBytes, kPlain, mk, mq, p, h->g_v);
   SAGA_CASE(64, 16) SAGA_CASE(64, 32) SAGA_CASE(64, 48) SAGA_CASE(64, 64)
   SAGA_CASE(128, 16) SAGA_CASE(128, 32) SAGA_CASE(128, 48) SAGA_CASE(128, 64)
 #undef SAGA_CASE
@@ -361,6 +386,46 @@ __global__ void selftest_wait_kernel(int* status) {
     volatile int never = 0;
     if (!mbar_wait(b, 0, &never)) atomicOr(status, 0x2 /* SAGA_STATUS_TIMEOUT */);
   }
+}
+
+// Group-shared selection: S2-S4 per value-head group (a programmatic dependent
+// of the group variant of the score pass).
+int launch_group(saga_ctx* h, const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* seq_lens, int N, int32_t* sel_idx, float* sel_stat,
+                 float* sel_logit, void* out) {
+  GroupParams p;
+  p.cand_mask = h->cand_mask;
+  p.mask_stride = h->mask_stride;
+  p.zkey = reinterpret_cast<uint32_t*>(h->z);
+  p.z_stride = h->z_stride;
+  p.gstat = h->gstat;
+  p.seq_lens = seq_lens;
+  p.h_q = h->h_q;
+  p.h_k = h->h_k;
+  p.g = h->g;
+  p.h_v = h->h_v;
+  p.g_v = h->g_v;
+  p.L_max = h->max_seq_len;
+  p.N = N;
+  p.cand_cap = kTopnCap;
+  p.lse_part = h->lse_part;
+  p.m_ref = h->m_ref;
+  p.t_lo = h->t_lo;
+  p.sel_idx = sel_idx;
+  p.sel_stat = sel_stat;
+  p.sel_logit = sel_logit;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.scale = h->scale;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = h->status;
+  const dim3 grid(h->batch * h->h_v);
+  constexpr size_t smem = TopnLayout<kTopnSelNarrow>::kBytes;
+  const cudaError_t e = (h->d == 64)
+      ? launch(h, group_kernel<64>, grid, dim3(kTopnThreads), smem, kPdl, p)
+      : launch(h, group_kernel<128>, grid, dim3(kTopnThreads), smem, kPdl, p);
+  return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
 int check_heads(saga_ctx* h, int h_q, int h_k, int h_v, int d) {
@@ -511,10 +576,14 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->mask_stride = h->z_stride / 32;
   const size_t mask_bytes = rows * static_cast<size_t>(h->mask_stride) * 4;
   const size_t samp_bytes = rows * static_cast<size_t>(kSampleSize) * 4;
+  // group-shared selection: statistic keys per value-head row, and s at the selection
+  const size_t rows_v = static_cast<size_t>(max_batch) * h_v;
+  const size_t gstat_bytes = rows_v * static_cast<size_t>(h->z_stride) * 4;
+  const size_t gsel_bytes = rows_v * static_cast<size_t>(max_N) * 4;
   const size_t total = al(z_bytes) + 2 * al(stat_bytes) + 2 * al(sel_bytes) + al(256) +
                        2 * al(qo_bytes) + al(static_cast<size_t>(max_batch) * 4) +
                        al(part_bytes) + 2 * al(stat_bytes) + al(mask_bytes) + al(samp_bytes) +
-                       al(stat_bytes) + al(mask_bytes);
+                       al(stat_bytes) + al(mask_bytes) + al(gstat_bytes) + al(gsel_bytes);
   if (cudaMalloc(&h->ws, total) != cudaSuccess) { delete h; return SAGA_ERR_CUDA; }
   uint8_t* w = static_cast<uint8_t*>(h->ws);
   h->z = reinterpret_cast<float*>(w); w += al(z_bytes);
@@ -532,7 +601,9 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->samp = reinterpret_cast<float*>(w); w += al(samp_bytes);
   h->t_lo = reinterpret_cast<float*>(w); w += al(stat_bytes);
   h->m_ref = reinterpret_cast<float*>(w); w += al(stat_bytes);
-  h->lse_part = reinterpret_cast<float*>(w);
+  h->lse_part = reinterpret_cast<float*>(w); w += al(mask_bytes);
+  h->gstat = reinterpret_cast<uint32_t*>(w); w += al(gstat_bytes);
+  h->gsel_stat = reinterpret_cast<float*>(w);
   h->scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
   if (cudaMemset(h->stat_min, 0xFF, stat_bytes) != cudaSuccess ||
       cudaMemset(h->counter, 0x00, stat_bytes) != cudaSuccess ||
@@ -590,6 +661,31 @@ int saga_atopn_step(saga_handle h, const void* q, const void* k_cache, const voi
   if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
   return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit, kModeStep,
                      const_cast<float*>(log_tau));
+}
+
+int saga_group_attn(saga_handle h, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* seq_lens, int h_q, int h_k, int h_v, int head_dim, int N,
+                    void* out, int32_t* sel_idx, float* sel_stat, float* sel_logit) {
+  if (!h) return SAGA_ERR_INVALID_ARG;
+  if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  if (!q || !k_cache || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
+  if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
+  // value groups inside key groups, every head of a key group in one epilogue warp,
+  // the weights of N x g_v in the key list's shared memory
+  if (h->h_v % h->h_k != 0 || h->npad > 32 || h->g_v > kGroupMaxGv || N > kGroupMaxN ||
+      N * h->g_v > kTopnCap || !use_candidates(h, N))
+    return SAGA_ERR_UNSUPPORTED;
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return SAGA_ERR_CUDA;
+  int32_t* si = sel_idx ? sel_idx : h->sel_idx;
+  float* ss = sel_stat ? sel_stat : h->gsel_stat;
+  float* sl = sel_logit ? sel_logit : h->sel_logit;
+  int rc;
+  if ((rc = launch_bounds(h, q, k_cache, seq_lens, N, true))) return rc;
+  if ((rc = launch_score(h, q, k_cache, seq_lens, h->z, h->z_stride, false, true, true, true)))
+    return rc;
+  return launch_group(h, q, k_cache, v_cache, seq_lens, N, si, ss, sl, out);
 }
 
 int saga_decode_selftest_timeout(saga_handle h) {

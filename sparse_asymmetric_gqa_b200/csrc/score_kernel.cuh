@@ -167,10 +167,16 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // order, to the row's z slots [32c, 32c + popcount).  No atomics on the data
 // path: every chunk has its own slots.
 // kLse (candidate mode only): the chunk sums of exp(z - m_ref) go to lse_part.
-template <int D, int NPAD, bool kCand, bool kLse = false>
+// kGroup (with kCand and kLse; g <= 32): candidates are kept per value-head group
+// of g_v query heads (group-shared selection): a position passes for its group
+// when any head of the group passes its own bound, and then all g_v of its keys
+// are stored.  Group row r = b * h_v + (kh * g) / g_v + v' takes the z rows
+// [r * g_v, (r + 1) * g_v) as one area: chunk c's passing positions, in position
+// order, at [32 c g_v, ...), g_v keys each; its masks go to cand_mask row r.
+template <int D, int NPAD, bool kCand, bool kLse = false, bool kGroup = false>
 __global__ void __launch_bounds__(kScoreThreads, 1)
 score_kernel(const __grid_constant__ CUtensorMap tmap_k,
-             const __grid_constant__ CUtensorMap tmap_q, const ScoreParams p) {
+             const __grid_constant__ CUtensorMap tmap_q, const ScoreParams p, const int g_v) {
   using S = ScoreShape<D, NPAD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -421,6 +427,41 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int chunk = c.t * (kTileM / 32) + quad;
           uint32_t* kslot = reinterpret_cast<uint32_t*>(p.z) + static_cast<long long>(row0) * p.z_stride + chunk * 32;
           uint32_t my_m = 0u;
+          if constexpr (kGroup) {
+            static_assert(!kGroup || (kCand && kLse), "groups come with candidates and sums");
+            // h0 = 0 and H >= g here: this lane holds every head of the key group
+            float zk[H];
+            uint32_t pm = 0u;                  // bit e: head e passes its bound
+#pragma unroll
+            for (int e = 0; e < H; ++e) {
+              const float zz = __fadd_rn(__fmul_rn(acc[e], p.scale), 0.0f);
+              zk[e] = zz;
+              const float a = zz - mr[e];
+              ls[e] += (valid && e < p.g) ? (a > kLseMaxExp ? INFINITY : __expf(a)) : 0.0f;
+              pm |= (valid && e < p.g && zz >= tl[e]) ? (1u << e) : 0u;
+            }
+            const int grow0 = c.b * (p.h_q / g_v) + (c.kh * p.g) / g_v;   // first group row
+#pragma unroll
+            for (int e = 0; e < H; ++e) {
+              if (e < p.g) {
+                const int ge = e / g_v, eo = e - ge * g_v;
+                const uint32_t gm = static_cast<uint32_t>(((1ull << g_v) - 1ull) << (ge * g_v));
+                const bool take = (pm & gm) != 0u;
+                const uint32_t m = __ballot_sync(0xffffffffu, take);
+                if (eo == 0 && lane == ge) my_m = m;
+                if (take) {
+                  uint32_t* gslot = reinterpret_cast<uint32_t*>(p.z) +
+                      static_cast<long long>(grow0 + ge) * g_v * p.z_stride +
+                      static_cast<long long>(chunk) * 32 * g_v;
+                  st_global_hint(gslot + __popc(m & lt) * g_v + eo, ordered_key(zk[e]), pol_z);
+                }
+              }
+            }
+            const int ng = p.g / g_v;
+            if (lane < ng && chunk * 32 < c.Lb)                   // lane v': group v''s mask
+              st_global_hint(p.cand_mask + static_cast<long long>(grow0 + lane) * p.mask_stride + chunk,
+                             my_m, pol_z);
+          } else {
 #pragma unroll
           for (int e = 0; e < H; ++e) {
             // fp32 dot product, then one fp32 scale; -0 canonicalised to +0.
@@ -438,6 +479,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           if (lane < H && h0 + lane < p.g && chunk * 32 < c.Lb)   // lane e: head e's mask
             st_global_hint(p.cand_mask + static_cast<long long>(row0 + lane) * p.mask_stride + chunk, my_m, pol_z);
+          }
           if (lse && chunk * 32 < c.Lb) {
             if (ls_chunk < 0) {                  // the piece's first chunk takes its total
               ls_chunk = chunk;

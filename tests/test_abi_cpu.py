@@ -68,6 +68,8 @@ def test_null_handle_rejected(lib):
         _lib.SAGA_ERR_INVALID_ARG
     assert lib.saga_decode_free(None) == _lib.SAGA_ERR_INVALID_ARG
     assert lib.saga_decode_selftest_timeout(None) == _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_group_attn(None, None, None, None, None, 1, 1, 1, 64, 1, None, None, None,
+                               None) == _lib.SAGA_ERR_INVALID_ARG
     assert lib.saga_atopn_calibrate(None, None, None, None, None, 1, 1, 1, 64, 1, None, None,
                                     None, None) == _lib.SAGA_ERR_INVALID_ARG
     assert lib.saga_atopn_step(None, None, None, None, None, 1, 1, 1, 64, 1, None, None,
