@@ -24,7 +24,6 @@ import io
 import json
 import math
 import os
-import re
 import subprocess
 import sys
 import threading
@@ -37,7 +36,7 @@ import torch  # noqa: E402
 
 METRIC = "decode-attn tokens/sec and achieved HBM GB/s (% of B200 roofline) at 32K ctx"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "score_kernel_qwen32k.md")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "score_kernel_qwen32k.json")
 SCORE_SOURCES = [os.path.join(ROOT, "sparse_asymmetric_gqa_b200", "csrc", f)
                  for f in ("score_kernel.cuh", "ptx.cuh")]
 
@@ -52,6 +51,10 @@ def parse_args():
     ap.add_argument("--impl", choices=["saga", "reference"], default="saga")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--workload", default="qwen32k",
+                    choices=["qwen32k", "dense_llama", "llama_ragged", "sweep"],
+                    help="qwen32k: the headline line (default); the others print one line of "
+                         "per-call throughput for that workload (the sweep: one line, 27 points)")
     ap.add_argument("--layers", type=int, default=None,
                     help="layers per step (default: the workload's 28); fewer only for small "
                          "profiling captures, never for a reported number")
@@ -109,17 +112,16 @@ def score_source_hash():
 
 
 def profiled_traffic():
-    """DRAM bytes per score-kernel launch from the committed ncu summary, or
-    None if the kernel source changed since it was captured."""
+    """DRAM bytes per score-kernel launch from the committed ncu capture's JSON
+    record, or None if the kernel source changed since it was captured."""
     try:
-        text = open(PROFILE_SUMMARY).read()
-    except OSError:
+        with open(PROFILE_TRAFFIC) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != score_source_hash():
+    if rec.get("source_sha256") != score_source_hash():
         return None
-    return float(m_bytes.group(1))
+    return float(rec["dram_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -285,6 +287,99 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------------------- CUDA leg
 
+def time_workload(spec, dev, steps, warmup, flush):
+    """Device time of one decode call of ``spec`` through SagaDecoder.attn: a CUDA
+    graph of the call, replayed ``steps`` times after ``warmup``, with L2 flushed
+    (a 256 MB write) before every replay and CUDA events around the replay only."""
+    from sparse_asymmetric_gqa_b200 import SagaDecoder, workload
+    x = workload.make_inputs(spec, layer=0, device=dev)
+    B = spec.batch
+    out = torch.empty(B, spec.h_q, spec.head_dim, dtype=torch.bfloat16, device=dev)
+    dec = SagaDecoder(B, spec.seq_len, spec.h_q, spec.h_k, spec.h_v, spec.head_dim, spec.N,
+                      device=dev)
+    dec.attn(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=out)
+    status = dec.status()
+    if status & 0xFF:
+        raise RuntimeError(f"{spec.name}: device status 0x{status:x}")
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        dec.attn(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=out)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    n0 = dec.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dec.attn(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=out)
+    launches = dec.launch_count() - n0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for _ in range(max(warmup, 3)):
+        flush.fill_(1.0)
+        graph.replay()
+    for a, b in ev:
+        flush.fill_(1.0)
+        a.record()
+        graph.replay()
+        b.record()
+    torch.cuda.synchronize(dev)
+    times = sorted(a.elapsed_time(b) for a, b in ev)
+    lens = [int(v) for v in x.seq_lens.tolist()]
+    k_bytes = sum(spec.h_k * Lb * spec.head_dim * 2 for Lb in lens)
+    v_bytes = sum(spec.h_v * min(spec.N, Lb) * spec.head_dim * 2 for Lb in lens)
+    del graph, dec, x
+    torch.cuda.empty_cache()
+    return {"ms_mean": sum(times) / len(times), "ms_median": times[len(times) // 2],
+            "launches": launches, "k_bytes": k_bytes, "v_bytes_model": v_bytes}
+
+
+def run_workloads(args, rank, world, local):
+    """One JSON line of per-call throughput for a workload other than the headline."""
+    from sparse_asymmetric_gqa_b200 import workload
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    if args.workload == "sweep":
+        specs = workload.sweep_specs()
+    else:
+        specs = [{"dense_llama": workload.DENSE_LLAMA, "llama_ragged": workload.LLAMA_RAGGED}[args.workload]]
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)     # 256 MB > 126 MB L2
+    peak, peak_src = measured_hbm_peak()
+    steps = max(3, min(args.steps, 20))
+    points = []
+    for spec in specs:
+        r = time_workload(spec, dev, steps, args.warmup, flush)
+        call_s = max_over_ranks(r["ms_mean"], world) / 1e3
+        gbs = (r["k_bytes"] + r["v_bytes_model"]) / call_s / 1e9
+        points.append({
+            "workload": spec.name, "batch": spec.batch, "seq_len": spec.seq_len, "N": spec.N,
+            "h_q": spec.h_q, "h_k": spec.h_k, "h_v": spec.h_v, "head_dim": spec.head_dim,
+            "ragged": spec.ragged, "tokens_per_s": world * spec.batch / call_s,
+            "calls_per_s": world / call_s, "ms_per_call": call_s * 1e3,
+            "ms_per_call_median": r["ms_median"], "gpu_launches_per_call": r["launches"],
+            "model_bytes_per_call": r["k_bytes"] + r["v_bytes_model"], "achieved_gbs": gbs,
+            "frac": gbs / peak,
+        })
+    if rank != 0:
+        return
+    head = points[0] if len(points) == 1 else None
+    line = {
+        "metric": "decode-attn tokens/sec and achieved HBM GB/s (% of B200 roofline)",
+        "workload": args.workload,
+        "value": head["tokens_per_s"] if head else None,
+        "unit": "tokens/s (one attention layer per call)",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "timing": "CUDA graph of one call, CUDA events around each replay, 256 MB L2 flush "
+                  "before each replay (outside the events)",
+        "roofline_model": "K cache over valid positions + N V rows per value head, at the "
+                          "measured copy bandwidth",
+        "peak_gbs": peak, "peak_source": peak_src,
+        "points": points,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_saga(args, rank, world, local):
     from sparse_asymmetric_gqa_b200 import SagaDecoder, workload
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
@@ -382,7 +477,17 @@ def run_saga(args, rank, world, local):
     p1.record()
     torch.cuda.synchronize(dev)
     prof_ms = max_over_ranks(p0.elapsed_time(p1), world)
-    score_ms, call_ms, n_prof = dec.profile_read()     # the last replay's events
+    # the events of one replay at a time (each read returns the last replay's), summed
+    # over up to 10 replays
+    score_ms = call_ms = 0.0
+    n_prof = 0
+    for _ in range(max(1, min(args.steps, 10))):
+        pgraph.replay()
+        torch.cuda.synchronize(dev)
+        s_ms, c_ms, n_c = dec.profile_read()
+        score_ms += s_ms
+        call_ms += c_ms
+        n_prof += n_c
 
     # ---- end to end through the host-buffer entry point (q in, out back, per layer)
     pin_q = [x.q.cpu().pin_memory() for x in layers]
@@ -454,6 +559,40 @@ def run_saga(args, rank, world, local):
     barrier(world)
     a_ms = max_over_ranks(a0.elapsed_time(a1), world)
     a_status = dec.status()
+
+    # ---- group-shared selection (one position set per value head), graphed and
+    # timed like the headline on the same caches and queries
+    def step_group():
+        for x, o in zip(layers, outs):
+            dec.group_attn(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=o)
+
+    step_group()
+    g_status = dec.status()
+    if g_status & 0xFF:
+        raise RuntimeError(f"device status 0x{g_status:x} in the group-shared step")
+    with torch.cuda.stream(side):
+        step_group()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    n2 = dec.launch_count()
+    ggraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ggraph):
+        step_group()
+    g_launches = dec.launch_count() - n2
+    for _ in range(max(args.warmup, 3)):
+        ggraph.replay()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    for _ in range(args.steps):
+        ggraph.replay()
+    g1.record()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    g_ms = max_over_ranks(g0.elapsed_time(g1), world)
+    g_status = dec.status()
     if clocks:
         clocks.stop()
 
@@ -469,7 +608,8 @@ def run_saga(args, rank, world, local):
     step_s = ms_max / 1e3 / args.steps
     value = world * B / step_s * L / spec.layers     # tokens of the full 28-layer model
     score_avg_s = score_ms / 1e3 / max(n_prof, 1)
-    call_avg_s = call_ms / 1e3 / max(n_prof, 1)
+    call_avg_s = step_s / L                         # per call, from the headline graph
+    prof_call_avg_s = call_ms / 1e3 / max(n_prof, 1)
     achieved = k_bytes / score_avg_s / 1e9
     call_gbs = model_bytes / call_avg_s / 1e9
     traffic = profiled_traffic()
@@ -489,6 +629,7 @@ def run_saga(args, rank, world, local):
         "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps,
         "ms_per_step_median": median_ms,
+        "calls_per_s": world * L / step_s,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -515,7 +656,10 @@ def run_saga(args, rank, world, local):
             "model_bytes_per_call": model_bytes, "avg_call_us": call_avg_s * 1e6,
             "achieved": call_gbs, "frac": call_gbs / peak, "unit": "GB/s",
             "model": "K cache over valid positions + N V rows per value head",
+            "source": "headline graph: ms_per_step / 28 calls",
+            "profiled_graph_avg_call_us": prof_call_avg_s * 1e6,
             "profiled_graph_ms_per_step": prof_ms / args.steps,
+            "profiled_replays_averaged": n_prof // max(L, 1),
             "v_bytes_per_query_head_model": v_bytes_per_head,
             "v_bytes_unique_rows_measured": v_bytes_unique,
         },
@@ -550,6 +694,16 @@ def run_saga(args, rank, world, local):
             "kept_per_row_mean": float(a_kept.mean()), "kept_per_row_max": int(a_kept.max()),
             "robust_path_seen": bool(a_status & 0x200),
         },
+        "group_select": {
+            "what": "group-shared selection (saga_group_attn): one set of N positions per value "
+                    "head from the summed softmax probabilities of its query heads, each head's "
+                    "own softmax over it; a different selection rule from the headline's",
+            "value": world * B / (g_ms / 1e3 / args.steps) * L / spec.layers,
+            "unit": "tokens/s", "ms_per_step": g_ms / args.steps,
+            "gpu_launches": g_launches * args.steps,
+            "v_bytes_per_call_model": v_bytes_model,
+            "robust_path_seen": bool(g_status & 0x200),
+        },
     }
     print(json.dumps(line), flush=True)
 
@@ -560,6 +714,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload != "qwen32k":
+            run_workloads(args, rank, world, local)
         else:
             run_saga(args, rank, world, local)
     finally:

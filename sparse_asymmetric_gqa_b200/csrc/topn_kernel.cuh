@@ -65,7 +65,7 @@ constexpr int kTopnBinsPer = kTopnBins / kTopnThreads;   // digits owned by a th
 constexpr int kTopnPer = 16;                      // entries per thread per step of the ordered pass
 constexpr int kTopnStep = kTopnPer * kTopnThreads;
 constexpr int kTopnRound = 4;                     // chunks per thread per round of loads
-constexpr int kTopnMaxRun = 8;                    // chunks per thread on the shared-memory path
+constexpr int kTopnMaxRun = 16;                   // chunks per thread on the shared-memory path (rows <= 131072)
 constexpr int kTopnMaxD = 128;
 
 // Dynamic shared memory, in 32-bit words, for selection lists of up to kSel

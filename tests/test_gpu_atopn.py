@@ -282,3 +282,51 @@ def test_full_size_qwen_calibrate_and_step_sampled_rows():
     assert all(abs(n - spec.N) <= 2 for n in kept)
     assert torch.isfinite(s_out.float()).all()
     assert torch.isfinite(log_tau).all()
+
+
+@pytest.mark.parametrize("shift", [0.0, -1.5, 2.0])
+def test_step_keeps_an_upper_set_of_its_own_scores(shift):
+    # The step's compare, bit-exact against the GPU's own fp32 scores (the stage-wise
+    # score pass computes them with the same arithmetic): its logits are those scores
+    # exactly, and the kept positions are the first 2N in position order of
+    # {i : z_i >= t} for one threshold t, so no position before the last kept one
+    # with a score at or above the smallest kept score is left out.  log tau is
+    # shifted (0: as calibrated; < 0 keeps more, hitting the 2N capacity; > 0 keeps
+    # fewer), and rows below and above the candidate cap are both covered.  A long
+    # row whose threshold falls below its sampled bound is scored again on CUDA
+    # cores (INFO_ROBUST_PATH), with another summation order: the long rows of
+    # such a call are not compared bit for bit.
+    B, L, h_q, h_k, h_v, d, N = 2, 20000, 4, 1, 2, 128, 256
+    lens = [L, 5000]
+    inp = make_raw(71, B, L, lens, h_q, h_k, h_v, d)
+    dec = SagaDecoder(B, L, h_q, h_k, h_v, d, N)
+    dev = _dev(inp)
+    _, _, _, log_tau, st = calibrate(dec, *dev, N)
+    assert st & 0xFF == 0
+    _, idx, logit, st = step(dec, *dev, N, log_tau + shift)
+    assert st & 0xFF == 0
+    rescored = bool(st & _lib.SAGA_STATUS_INFO_ROBUST_PATH)
+    z = dec.score(dev[0], dev[1], dev[3]).cpu().numpy()
+    idx, logit = idx.cpu().numpy(), logit.cpu().numpy()
+    checked = 0
+    for b in range(B):
+        if rescored and lens[b] > 8192:
+            continue
+        for j in range(h_q):
+            what = f"shift {shift} ({b},{j})"
+            checked += 1
+            kept = idx[b, j][idx[b, j] >= 0]
+            n = kept.size
+            assert (idx[b, j, n:] == -1).all(), f"{what}: padding"
+            zr = z[b, j, :lens[b]]
+            np.testing.assert_array_equal(logit[b, j, :n], zr[kept], err_msg=what)
+            if n == 0:
+                continue
+            assert (np.diff(kept) > 0).all(), f"{what}: not ascending"
+            t_min = zr[kept].min()
+            left_out = np.ones(kept[-1] + 1, dtype=bool)
+            left_out[kept] = False
+            assert (zr[:kept[-1] + 1][left_out] < t_min).all(), f"{what}: a score >= the kept ones left out"
+            if n < 2 * N:                               # below capacity: nothing after the last one either
+                assert (zr[kept[-1] + 1:] < t_min).all(), f"{what}: a later score >= the kept ones left out"
+    assert checked >= h_q

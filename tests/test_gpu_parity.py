@@ -118,7 +118,7 @@ SWEEP_POINTS = ["qwen_sweep_b1_l128k_n2048", "qwen_sweep_b8_l32k_n1024",
 @pytest.mark.parametrize("name", SWEEP_POINTS)
 def test_sweep_points_sampled_rows(name):
     # Corners of the long-context sweep (Qwen shapes, 1% planted keys), inputs drawn
-    # on the device; rows of 128K positions take the slot path (INFO_ROBUST_PATH).
+    # on the device; rows of 128K positions fit the shared-memory candidate list.
     spec = SWEEP[name]
     inp = workload.make_inputs(spec, device="cuda")
     dec = SagaDecoder(spec.batch, spec.seq_len, spec.h_q, spec.h_k, spec.h_v, spec.head_dim, spec.N)
