@@ -262,8 +262,10 @@ SAGA_API int saga_decode_launch_count(saga_handle h, long long* count);
  * records become graph nodes, so every replay re-records them; the events
  * live until the handle is freed).  Disabling stops recording and keeps the
  * events.  saga_decode_profile_read synchronises and returns the summed
- * milliseconds and the number of calls recorded, then starts counting calls
- * from zero again. */
+ * milliseconds of the calls recorded since profiling was last enabled, and
+ * their number; it may be called after every replay of a graph that holds the
+ * records (each read gives that replay's times).  Enabling again starts
+ * counting calls from zero. */
 SAGA_API int saga_decode_profile(saga_handle h, int enable, int max_calls);
 SAGA_API int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms,
                              int* n_calls);

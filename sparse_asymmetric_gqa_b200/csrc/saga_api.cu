@@ -815,7 +815,6 @@ int saga_decode_profile_read(saga_handle h, double* score_ms, double* call_ms, i
   *score_ms = s;
   *call_ms = c;
   *n_calls = h->prof_n;
-  h->prof_n = 0;
   return SAGA_OK;
 }
 
