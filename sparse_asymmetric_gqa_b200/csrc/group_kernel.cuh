@@ -147,7 +147,7 @@ group_kernel(const GroupParams p) {
   // ---- 1: masks and per-head chunk sums; thread t owns chunks [c0, c1)
   const int cpt = (nch + kTopnThreads - 1) / kTopnThreads;
   const int c0 = min(nch, tid * cpt), c1 = min(nch, c0 + cpt);
-  const bool fits = cpt <= kTopnMaxRun;
+  const bool fits = cpt <= kTopnRun;
   uint32_t cnt = 0u;
   float lsum[kGroupMaxGv];
 #pragma unroll

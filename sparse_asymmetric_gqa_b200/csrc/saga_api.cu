@@ -158,6 +158,14 @@ int set_smem_attrs_once() {
     SAGA_TOPN_ATTR(64, kModeStep, kTopnSelNarrow) SAGA_TOPN_ATTR(128, kModeStep, kTopnSelNarrow)
     SAGA_TOPN_ATTR(64, kModeStep, kTopnSelMax) SAGA_TOPN_ATTR(128, kModeStep, kTopnSelMax)
 #undef SAGA_TOPN_ATTR
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
     rc = (e == cudaSuccess) ? 0 : 1;
   });
   return rc;
@@ -313,8 +321,11 @@ int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   constexpr size_t narrow = TopnLayout<kTopnSelNarrow>::kBytes, wide = TopnLayout<kTopnSelMax>::kBytes;
   cudaError_t e;
   if (mode == kModeExact)
-    e = (h->d == 64) ? launch(h, topn_kernel<64, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
-                     : launch(h, topn_kernel<128, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p);
+    e = h->max_seq_len > kTopnThreads * 32 * kTopnRun
+        ? ((h->d == 64) ? launch(h, topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun>, grid, block, narrow, kPdl, p)
+                        : launch(h, topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun>, grid, block, narrow, kPdl, p))
+        : ((h->d == 64) ? launch(h, topn_kernel<64, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
+                        : launch(h, topn_kernel<128, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p));
   else if (mode == kModeCalibrate)
     e = (h->d == 64) ? launch(h, topn_kernel<64, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
                      : launch(h, topn_kernel<128, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p);

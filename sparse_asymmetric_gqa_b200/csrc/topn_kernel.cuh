@@ -65,7 +65,8 @@ constexpr int kTopnBinsPer = kTopnBins / kTopnThreads;   // digits owned by a th
 constexpr int kTopnPer = 16;                      // entries per thread per step of the ordered pass
 constexpr int kTopnStep = kTopnPer * kTopnThreads;
 constexpr int kTopnRound = 4;                     // chunks per thread per round of loads
-constexpr int kTopnMaxRun = 16;                   // chunks per thread on the shared-memory path (rows <= 131072)
+constexpr int kTopnRun = 8;                       // chunks per thread on the shared-memory path (rows <= 65536)
+constexpr int kTopnLongRun = 16;                  // the long-row variant (rows <= 131072)
 constexpr int kTopnMaxD = 128;
 
 // Dynamic shared memory, in 32-bit words, for selection lists of up to kSel
@@ -435,7 +436,10 @@ __device__ void topn_rescore(const __nv_bfloat16* q, const __nv_bfloat16* keys, 
 }
 
 // kMode: a TopnMode; kSel: the layout's selection capacity (>= the list width p.cap).
-template <int D, int kMode, int kSel>
+// kRun: chunks per thread the shared-memory path takes (kTopnRun, or kTopnLongRun
+// for caches of more than 65536 positions; the longer variant costs the short
+// rows a few microseconds).
+template <int D, int kMode, int kSel, int kRun = kTopnRun>
 __global__ void __launch_bounds__(kTopnThreads, 2)
 topn_kernel(const TopnParams p) {
   using Lay = TopnLayout<kSel>;
@@ -482,12 +486,12 @@ topn_kernel(const TopnParams p) {
   // (and the chunk sums)
   const int cpt = (nch + kTopnThreads - 1) / kTopnThreads;
   const int c0 = min(nch, tid * cpt), c1 = min(nch, c0 + cpt);
-  const bool fits = cpt <= kTopnMaxRun;
-  uint32_t run_mask[kTopnMaxRun];
-  float run_sum[kTopnMaxRun];
+  const bool fits = cpt <= kRun;
+  uint32_t run_mask[kRun];
+  float run_sum[kRun];
   uint4 sec[kTopnRound][2];
 #pragma unroll
-  for (int u = 0; u < kTopnMaxRun; ++u) {
+  for (int u = 0; u < kRun; ++u) {
     run_mask[u] = (c0 + u < c1) ? __ldcg(mrow + c0 + u) : 0u;
     run_sum[u] = (sums && c0 + u < c1) ? __ldcg(lrow + c0 + u) : 0.0f;
   }
@@ -500,9 +504,9 @@ topn_kernel(const TopnParams p) {
   uint32_t cnt = 0u;
   float lsum = 0.0f;
 #pragma unroll
-  for (int u = 0; u < kTopnMaxRun; ++u) { cnt += __popc(run_mask[u]); lsum += run_sum[u]; }
+  for (int u = 0; u < kRun; ++u) { cnt += __popc(run_mask[u]); lsum += run_sum[u]; }
   if (!fits)
-    for (int c = c0 + kTopnMaxRun; c < c1; ++c) {
+    for (int c = c0 + kRun; c < c1; ++c) {
       cnt += __popc(__ldcg(mrow + c));
       if (sums) lsum += __ldcg(lrow + c);
     }
@@ -522,7 +526,7 @@ topn_kernel(const TopnParams p) {
   auto gather_list = [&]() {
     uint32_t o = off;
 #pragma unroll
-    for (int u0 = 0; u0 < kTopnMaxRun; u0 += kTopnRound) {
+    for (int u0 = 0; u0 < kRun; u0 += kTopnRound) {
       if (u0 >= cpt) break;                      // uniform
       if (u0 > 0) {                              // rows longer than kTopnRound chunks per thread
 #pragma unroll
