@@ -375,6 +375,9 @@ def run_workloads(args, rank, world, local):
         "roofline_model": "K cache over valid positions + N V rows per value head, at the "
                           "measured copy bandwidth",
         "peak_gbs": peak, "peak_source": peak_src,
+        "parity": "checked by the GPU tests, not here: tests/test_gpu_parity.py (these workloads' "
+                  "sampled rows, four sweep corners), tests/test_gpu_full_layer.py (every row of "
+                  "a Qwen 32K and a ragged Llama layer)",
         "points": points,
     }
     print(json.dumps(line), flush=True)
@@ -656,6 +659,8 @@ def run_saga(args, rank, world, local):
             "model_bytes_per_call": model_bytes, "avg_call_us": call_avg_s * 1e6,
             "achieved": call_gbs, "frac": call_gbs / peak, "unit": "GB/s",
             "model": "K cache over valid positions + N V rows per value head",
+            "shipped_path_reads": "N V rows per query head (v_bytes_per_query_head_model); the "
+                                  "per-value-head byte model is what the group-shared path reads",
             "source": "headline graph: ms_per_step / 28 calls",
             "profiled_graph_avg_call_us": prof_call_avg_s * 1e6,
             "profiled_graph_ms_per_step": prof_ms / args.steps,
