@@ -37,6 +37,11 @@ constexpr int kGroupMaxGv = 8;            // query heads per value head
 constexpr int kGroupMaxN = 1024;          // N * g_v weights live in the key list's region
 constexpr float kGroupMargin = 1e-4f;     // relative margin of the completeness check
 constexpr int kGroupBatch = 16;           // value rows per warp per round of loads
+constexpr int kGroupBlock = 4;            // kept positions whose keys are loaded together
+// Candidates of a group held in shared memory: the union of g_v heads' lists
+// (one CTA per group, so one CTA per SM costs nothing here).
+constexpr int kGroupCap = 16384;
+using GroupLayout = TopnLayout<kTopnSelNarrow, kGroupCap>;
 
 struct GroupParams {
   const uint32_t* cand_mask;    // [B*h_v][mask_stride] positions kept for the group
@@ -105,7 +110,7 @@ __device__ __forceinline__ long long group_key_at(const uint32_t* mrow, int pos,
 template <int D>
 __global__ void __launch_bounds__(kTopnThreads, 2)
 group_kernel(const GroupParams p) {
-  using Lay = TopnLayout<kTopnSelNarrow>;
+  using Lay = GroupLayout;
   extern __shared__ __align__(16) uint32_t group_smem[];
   uint32_t* s_key = group_smem + Lay::kOffKey;       // candidate keys of s; then the weights
   int32_t* s_pos = reinterpret_cast<int32_t*>(group_smem + Lay::kOffPos);   // positions; then P.V partials
@@ -228,23 +233,36 @@ group_kernel(const GroupParams p) {
       __syncthreads();                           // srow is complete for the whole CTA
       listp = false;
     } else {
-      listp = C <= static_cast<uint32_t>(kTopnCap) && fits;
+      listp = C <= static_cast<uint32_t>(kGroupCap) && fits;
       uint32_t o = off;
+      // a chunk's kept positions hold their keys at consecutive slots: the keys of
+      // kGroupBlock positions (all heads) are loaded before any of them is used
       for (int c = c0; c < c1; ++c) {
         uint32_t m = __ldcg(mrow + c);
         const int n_c = __popc(m);
-        for (int k = 0; k < n_c; ++k) {
-          const int pos = c * 32 + (__ffs(m) - 1);
-          m &= m - 1u;
-          float s = 0.0f;
+        const uint32_t* ac = area + static_cast<long long>(c) * 32 * g_v;
+        for (int k0 = 0; k0 < n_c; k0 += kGroupBlock) {
+          uint32_t kv[kGroupBlock][kGroupMaxGv];
 #pragma unroll
-          for (int e = 0; e < kGroupMaxGv; ++e)
-            if (e < g_v)
-              s += expf(key_to_float(__ldcg(area + (static_cast<long long>(c) * 32 + k) * g_v + e)) - lse[e]);
-          const uint32_t key = ordered_key(s);
-          srow[c * 32 + k] = key;
-          if (listp) { s_key[o] = key; s_pos[o] = pos; }
-          ++o;
+          for (int u = 0; u < kGroupBlock; ++u)
+#pragma unroll
+            for (int e = 0; e < kGroupMaxGv; ++e)
+              kv[u][e] = (k0 + u < n_c && e < g_v) ? __ldcg(ac + (k0 + u) * g_v + e) : 0u;
+#pragma unroll
+          for (int u = 0; u < kGroupBlock; ++u) {
+            if (k0 + u < n_c) {
+              const int pos = c * 32 + (__ffs(m) - 1);
+              m &= m - 1u;
+              float s = 0.0f;
+#pragma unroll
+              for (int e = 0; e < kGroupMaxGv; ++e)
+                if (e < g_v) s += expf(key_to_float(kv[u][e]) - lse[e]);
+              const uint32_t key = ordered_key(s);
+              srow[c * 32 + k0 + u] = key;
+              if (listp) { s_key[o] = key; s_pos[o] = pos; }
+              ++o;
+            }
+          }
         }
       }
       __syncthreads();

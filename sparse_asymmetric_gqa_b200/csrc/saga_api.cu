@@ -145,10 +145,10 @@ int set_smem_attrs_once() {
                                static_cast<int>(sizeof(SelectSmem)));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(group_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
+                               static_cast<int>(GroupLayout::kBytes));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(group_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
+                               static_cast<int>(GroupLayout::kBytes));
 #define SAGA_TOPN_ATTR(D, M, S)                                                                   \
   if (e == cudaSuccess)                                                                           \
     e = cudaFuncSetAttribute(topn_kernel<D, M, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
@@ -432,7 +432,7 @@ int launch_group(saga_ctx* h, const void* q, const void* k_cache, const void* v_
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = h->status;
   const dim3 grid(h->batch * h->h_v);
-  constexpr size_t smem = TopnLayout<kTopnSelNarrow>::kBytes;
+  constexpr size_t smem = GroupLayout::kBytes;
   const cudaError_t e = (h->d == 64)
       ? launch(h, group_kernel<64>, grid, dim3(kTopnThreads), smem, kPdl, p)
       : launch(h, group_kernel<128>, grid, dim3(kTopnThreads), smem, kPdl, p);

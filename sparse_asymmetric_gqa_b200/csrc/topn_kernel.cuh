@@ -69,14 +69,15 @@ constexpr int kTopnRun = 8;                       // chunks per thread on the sh
 constexpr int kTopnLongRun = 16;                  // the long-row variant (rows <= 131072)
 constexpr int kTopnMaxD = 128;
 
-// Dynamic shared memory, in 32-bit words, for selection lists of up to kSel
-// entries; every region starts on a 16-byte boundary.  (90 KB for kSel = 2048:
-// two CTAs per SM; the wide layout of a step with N > 1024 takes 106 KB.)
-template <int kSel>
+// Dynamic shared memory, in 32-bit words, for candidate lists of up to kCap
+// and selection lists of up to kSel entries; every region starts on a 16-byte
+// boundary.  (90 KB for kSel = 2048: two CTAs per SM; the wide layout of a step
+// with N > 1024 takes 106 KB.)
+template <int kSel, int kCap = kTopnCap>
 struct TopnLayout {
-  static constexpr int kOffKey = 0;                             // [kTopnCap] candidate keys
-  static constexpr int kOffPos = kOffKey + kTopnCap;            // [kTopnCap] candidate positions
-  static constexpr int kOffSelPos = kOffPos + kTopnCap;         // [kSel] selected positions
+  static constexpr int kOffKey = 0;                             // [kCap] candidate keys
+  static constexpr int kOffPos = kOffKey + kCap;                // [kCap] candidate positions
+  static constexpr int kOffSelPos = kOffPos + kCap;             // [kSel] selected positions
   static constexpr int kOffSelW = kOffSelPos + kSel;            // [kSel] softmax weights
   static constexpr int kOffHist = kOffSelW + kSel;              // [kTopnBins]; P.V partials [warps][D]
   static constexpr int kOffScan = kOffHist + kTopnBins;         // [kTopnWarps]
