@@ -37,7 +37,7 @@ constexpr int kGroupMaxGv = 8;            // query heads per value head
 constexpr int kGroupMaxN = 1024;          // N * g_v weights live in the key list's region
 constexpr float kGroupMargin = 1e-4f;     // relative margin of the completeness check
 constexpr int kGroupBatch = 16;           // value rows per warp per round of loads
-constexpr int kGroupBlock = 4;            // kept positions whose keys are loaded together
+constexpr int kGroupBlock = 8;            // kept positions whose keys are loaded together
 // Candidates of a group held in shared memory: the union of g_v heads' lists
 // (one CTA per group, so one CTA per SM costs nothing here).
 constexpr int kGroupCap = 16384;
@@ -300,23 +300,33 @@ group_kernel(const GroupParams p) {
   __syncthreads();                               // s_selpos complete; s_key / s_pos free
 
   // ---- 5: each head's logits at the set, softmax weights, and one P.V pass
+  // one lookup of a position's key slot serves all g_v heads (head e's key at +e)
   float zmax[kGroupMaxGv], wtot[kGroupMaxGv];
+  uint32_t khi[kGroupMaxGv];
+#pragma unroll
+  for (int e = 0; e < kGroupMaxGv; ++e) { zmax[e] = 0.0f; wtot[e] = 0.0f; khi[e] = 0u; }
+  float* lo0 = p.sel_logit + (static_cast<long long>(b) * p.h_q + j0) * N;
+#pragma unroll 4
+  for (int i = tid; i < static_cast<int>(n_b); i += kTopnThreads) {
+    const long long at = group_key_at(mrow, s_selpos[i], g_v, 0, all);
+    uint32_t kk[kGroupMaxGv];
+#pragma unroll
+    for (int e = 0; e < kGroupMaxGv; ++e) kk[e] = e < g_v ? __ldcg(area + at + e) : 0u;
+#pragma unroll
+    for (int e = 0; e < kGroupMaxGv; ++e) {
+      if (e < g_v) {
+        const float z = key_to_float(kk[e]);
+        lo0[static_cast<long long>(e) * N + i] = z;
+        s_w[i * g_v + e] = z;
+        khi[e] = max(khi[e], kk[e]);
+      }
+    }
+  }
 #pragma unroll
   for (int e = 0; e < kGroupMaxGv; ++e) {
-    zmax[e] = 0.0f;
-    wtot[e] = 0.0f;
     if (e < g_v) {
-      float* lo = p.sel_logit + (static_cast<long long>(b) * p.h_q + j0 + e) * N;
-      uint32_t hi = 0u;
-      for (int i = tid; i < static_cast<int>(n_b); i += kTopnThreads) {
-        const uint32_t key = __ldcg(area + group_key_at(mrow, s_selpos[i], g_v, e, all));
-        const float z = key_to_float(key);
-        lo[i] = z;
-        s_w[i * g_v + e] = z;
-        hi = max(hi, key);
-      }
-      for (int i = static_cast<int>(n_b) + tid; i < N; i += kTopnThreads) lo[i] = -INFINITY;
-      zmax[e] = key_to_float(topn_block_max(hi, s_scan));
+      for (int i = static_cast<int>(n_b) + tid; i < N; i += kTopnThreads) lo0[static_cast<long long>(e) * N + i] = -INFINITY;
+      zmax[e] = key_to_float(topn_block_max(khi[e], s_scan));
     }
   }
 #pragma unroll
