@@ -102,6 +102,20 @@ SAGA_API int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_le
                      int h_q, int h_k, int h_v, int head_dim, int max_N,
                      void* cuda_stream);
 
+/* As saga_decode_init, with keys (and queries) of width head_dim and values (and
+ * outputs) of width head_dim_v, each 64 or 128 ("More Value per Key" §5.2: keys
+ * narrower than values; the scale stays 1/sqrt(head_dim)).  On such a handle the
+ * head_dim argument of every call is the key width; q is [B][h_q][head_dim],
+ * k_cache [B][h_k][L_max][head_dim], v_cache [B][h_v][L_max][head_dim_v], out
+ * [B][h_q][head_dim_v], and saga_combine takes head_dim_v.  With head_dim_v !=
+ * head_dim only the exact decode step (saga_decode_attn*, candidate and score-row
+ * paths) and the stage-wise calls are supported: the stateful Atop-N calls and
+ * saga_group_attn return SAGA_ERR_UNSUPPORTED.  The workspace takes
+ * max(head_dim, head_dim_v) where the formula above has head_dim. */
+SAGA_API int saga_decode_init_kv(saga_handle* handle, int max_batch, int max_seq_len,
+                        int h_q, int h_k, int h_v, int head_dim, int head_dim_v, int max_N,
+                        void* cuda_stream);
+
 /* Set the batch B (1 <= B <= max_batch) used by later calls. */
 SAGA_API int saga_decode_set_batch(saga_handle h, int batch);
 

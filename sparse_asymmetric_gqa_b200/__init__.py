@@ -42,15 +42,18 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None, device=None):
 class SagaDecoder:
     """A handle of the library: fixed head layout and maximum sizes, one workspace.
 
-    Caches are [B, h, max_seq_len, head_dim] bf16 (h = h_k for keys, h_v for
+    head_dim_v (default head_dim) is the value and output width: keys may be
+    narrower (or wider) than values ("More Value per Key" §5.2).
+    Caches are [B, h, max_seq_len, width] bf16 (h = h_k for keys, h_v for
     values); ``seq_lens`` int32 [B] gives the valid positions of each row.
     """
 
     def __init__(self, max_batch: int, max_seq_len: int, h_q: int, h_k: int, h_v: int,
-                 head_dim: int, max_N: int, device=None):
+                 head_dim: int, max_N: int, device=None, head_dim_v=None):
         self.lib = load()
         self.max_batch, self.max_seq_len = max_batch, max_seq_len
         self.h_q, self.h_k, self.h_v, self.head_dim, self.max_N = h_q, h_k, h_v, head_dim, max_N
+        self.head_dim_v = head_dim if head_dim_v is None else head_dim_v
         self.batch = max_batch
         if device is None:
             self.device = torch.device("cuda", torch.cuda.current_device())
@@ -60,9 +63,9 @@ class SagaDecoder:
         self._h = ctypes.c_void_p()
         with torch.cuda.device(self.device):
             stream = torch.cuda.current_stream(self.device).cuda_stream
-            _lib.check("saga_decode_init", self.lib.saga_decode_init(
-                ctypes.byref(self._h), max_batch, max_seq_len, h_q, h_k, h_v, head_dim, max_N,
-                ctypes.c_void_p(stream)))
+            _lib.check("saga_decode_init_kv", self.lib.saga_decode_init_kv(
+                ctypes.byref(self._h), max_batch, max_seq_len, h_q, h_k, h_v, head_dim,
+                self.head_dim_v, max_N, ctypes.c_void_p(stream)))
 
     # ------------------------------------------------------------------ plumbing
     def _stream(self):
@@ -80,7 +83,7 @@ class SagaDecoder:
         if k_cache is not None:
             _need(k_cache, "k_cache", torch.bfloat16, (B, self.h_k, L, d), "cuda")
         if v_cache is not None:
-            _need(v_cache, "v_cache", torch.bfloat16, (B, self.h_v, L, d), "cuda")
+            _need(v_cache, "v_cache", torch.bfloat16, (B, self.h_v, L, self.head_dim_v), "cuda")
         if seq_lens is not None:
             _need(seq_lens, "seq_lens", torch.int32, (B,), "cuda")
 
@@ -90,8 +93,8 @@ class SagaDecoder:
         self._check_caches(q, k_cache, v_cache, seq_lens)
         B = self.batch
         if out is None:
-            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
-        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+            out = torch.empty(B, self.h_q, self.head_dim_v, dtype=torch.bfloat16, device=q.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim_v), "cuda")
         if sel_idx is not None:
             _need(sel_idx, "sel_idx", torch.int32, (B, self.h_q, N), "cuda")
         if sel_logit is not None:
@@ -114,8 +117,8 @@ class SagaDecoder:
         self._check_caches(q, k_cache, v_cache, seq_lens)
         B = self.batch
         if out is None:
-            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
-        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+            out = torch.empty(B, self.h_q, self.head_dim_v, dtype=torch.bfloat16, device=q.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim_v), "cuda")
         if sel_idx is not None:
             _need(sel_idx, "sel_idx", torch.int32, (B, self.h_v, N), "cuda")
         if sel_stat is not None:
@@ -139,10 +142,10 @@ class SagaDecoder:
         self._check_caches(q, k_cache, v_cache, seq_lens)
         B = self.batch
         if out is None:
-            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
+            out = torch.empty(B, self.h_q, self.head_dim_v, dtype=torch.bfloat16, device=q.device)
         if log_tau is None:
             log_tau = torch.empty(B, self.h_q, dtype=torch.float32, device=q.device)
-        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim_v), "cuda")
         _need(log_tau, "log_tau", torch.float32, (B, self.h_q), "cuda")
         if sel_idx is not None:
             _need(sel_idx, "sel_idx", torch.int32, (B, self.h_q, N), "cuda")
@@ -164,8 +167,8 @@ class SagaDecoder:
         self._check_caches(q, k_cache, v_cache, seq_lens)
         B = self.batch
         if out is None:
-            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=q.device)
-        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+            out = torch.empty(B, self.h_q, self.head_dim_v, dtype=torch.bfloat16, device=q.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim_v), "cuda")
         _need(log_tau, "log_tau", torch.float32, (B, self.h_q), "cuda")
         if sel_idx is not None:
             _need(sel_idx, "sel_idx", torch.int32, (B, self.h_q, 2 * N), "cuda")
@@ -182,7 +185,7 @@ class SagaDecoder:
         B = self.batch
         _need(q_host, "q_host", torch.bfloat16, (B, self.h_q, self.head_dim), "cpu")
         _need(seq_lens_host, "seq_lens_host", torch.int32, (B,), "cpu")
-        _need(out_host, "out_host", torch.bfloat16, (B, self.h_q, self.head_dim), "cpu")
+        _need(out_host, "out_host", torch.bfloat16, (B, self.h_q, self.head_dim_v), "cpu")
         self._check_caches(None, k_cache, v_cache, None)
         self._stream()
         _lib.check("saga_decode_attn_host", self.lib.saga_decode_attn_host(
@@ -230,12 +233,12 @@ class SagaDecoder:
         _need(sel_logit, "sel_logit", torch.float32, (B, self.h_q, N), "cuda")
         self._check_caches(None, None, v_cache, seq_lens)
         if out is None:
-            out = torch.empty(B, self.h_q, self.head_dim, dtype=torch.bfloat16, device=v_cache.device)
-        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim), "cuda")
+            out = torch.empty(B, self.h_q, self.head_dim_v, dtype=torch.bfloat16, device=v_cache.device)
+        _need(out, "out", torch.bfloat16, (B, self.h_q, self.head_dim_v), "cuda")
         self._stream()
         _lib.check("saga_combine", self.lib.saga_combine(
             self._h, _ptr(sel_idx), _ptr(sel_logit), _ptr(v_cache), _ptr(seq_lens),
-            self.h_q, self.h_v, self.head_dim, N, _ptr(out)))
+            self.h_q, self.h_v, self.head_dim_v, N, _ptr(out)))
         return out
 
     # ------------------------------------------------------------------ status

@@ -23,6 +23,7 @@ _I = ctypes.c_int
 # name -> (restype, argtypes)
 SIGNATURES = {
     "saga_decode_init": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _P]),
+    "saga_decode_init_kv": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "saga_decode_set_batch": (_I, [_P, _I]),
     "saga_decode_set_stream": (_I, [_P, _P]),
     "saga_decode_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),

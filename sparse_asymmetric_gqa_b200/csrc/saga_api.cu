@@ -81,6 +81,7 @@ struct saga_ctx {
   int device = 0;
   int num_sms = 0;
   int max_batch = 0, batch = 0, max_seq_len = 0, h_q = 0, h_k = 0, h_v = 0, d = 0, max_N = 0;
+  int dv = 0;                     // value and output width (d: the query and key width)
   int g = 0, g_v = 0, npad = 0;
   long long z_stride = 0;
   cudaStream_t stream = nullptr;
@@ -95,7 +96,7 @@ struct saga_ctx {
   __nv_bfloat16* q_stage = nullptr;
   __nv_bfloat16* out_stage = nullptr;
   int32_t* lens_stage = nullptr;
-  float scale = 0.0f;             // 1/sqrt(d) rounded to fp32
+  float scale = 0.0f;             // 1/sqrt(d) rounded to fp32 (d the key width)
   uint32_t* cand_mask = nullptr;  // candidate chunk masks [rows][mask_stride]
   long long mask_stride = 0;      // z_stride / 32
   float* samp = nullptr;          // sampled scores [rows][kSampleSize]
@@ -158,14 +159,16 @@ int set_smem_attrs_once() {
     SAGA_TOPN_ATTR(64, kModeStep, kTopnSelNarrow) SAGA_TOPN_ATTR(128, kModeStep, kTopnSelNarrow)
     SAGA_TOPN_ATTR(64, kModeStep, kTopnSelMax) SAGA_TOPN_ATTR(128, kModeStep, kTopnSelMax)
 #undef SAGA_TOPN_ATTR
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
+    // the exact kernel's other variants: long rows, and key widths other than the value width
+    for (const void* f : {reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun>),
+                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun>),
+                          reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnRun, 128>),
+                          reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun, 128>),
+                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnRun, 64>),
+                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun, 64>)})
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
     rc = (e == cudaSuccess) ? 0 : 1;
   });
   return rc;
@@ -257,6 +260,16 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
 }
 
+// The exact top-N kernel for value width DV and key width DK, with the 16-chunk
+// candidate path for caches of more than 65536 positions.
+template <int DV, int DK>
+cudaError_t launch_topn_exact(saga_ctx* h, dim3 grid, dim3 block, size_t smem, const TopnParams& p,
+                              bool long_rows) {
+  return long_rows
+      ? launch(h, topn_kernel<DV, kModeExact, kTopnSelNarrow, kTopnLongRun, DK>, grid, block, smem, kPdl, p)
+      : launch(h, topn_kernel<DV, kModeExact, kTopnSelNarrow, kTopnRun, DK>, grid, block, smem, kPdl, p);
+}
+
 // Candidate bounds for the n_target largest scores of each row: the sample
 // kernel (after the previous kernel in the stream) and the bound kernel (a
 // programmatic dependent of it); with ref, also the exp-sum references.
@@ -320,13 +333,13 @@ int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
   const dim3 block(kTopnThreads);
   constexpr size_t narrow = TopnLayout<kTopnSelNarrow>::kBytes, wide = TopnLayout<kTopnSelMax>::kBytes;
   cudaError_t e;
-  if (mode == kModeExact)
-    e = h->max_seq_len > kTopnThreads * 32 * kTopnRun
-        ? ((h->d == 64) ? launch(h, topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun>, grid, block, narrow, kPdl, p)
-                        : launch(h, topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun>, grid, block, narrow, kPdl, p))
-        : ((h->d == 64) ? launch(h, topn_kernel<64, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
-                        : launch(h, topn_kernel<128, kModeExact, kTopnSelNarrow>, grid, block, narrow, kPdl, p));
-  else if (mode == kModeCalibrate)
+  if (mode == kModeExact) {
+    const bool long_rows = h->max_seq_len > kTopnThreads * 32 * kTopnRun;
+    if (h->dv == 64 && h->d == 64) e = launch_topn_exact<64, 64>(h, grid, block, narrow, p, long_rows);
+    else if (h->dv == 128 && h->d == 128) e = launch_topn_exact<128, 128>(h, grid, block, narrow, p, long_rows);
+    else if (h->dv == 128) e = launch_topn_exact<128, 64>(h, grid, block, narrow, p, long_rows);
+    else e = launch_topn_exact<64, 128>(h, grid, block, narrow, p, long_rows);
+  } else if (mode == kModeCalibrate)
     e = (h->d == 64) ? launch(h, topn_kernel<64, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
                      : launch(h, topn_kernel<128, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p);
   else if (p.cap <= kTopnSelNarrow)
@@ -379,7 +392,7 @@ int launch_gather(saga_ctx* h, const int32_t* sel_idx, const float* sel_logit,
   p.status = h->status;
   const int slots = N < h->max_seq_len ? N : h->max_seq_len;
   const dim3 grid(h->batch * h->h_q, (slots + kGatherRows - 1) / kGatherRows);
-  const cudaError_t e = (h->d == 64)
+  const cudaError_t e = (h->dv == 64)
       ? launch(h, gather_kernel<64>, grid, dim3(kGatherThreads), 0, pdl ? kPdl : kPlain, p)
       : launch(h, gather_kernel<128>, grid, dim3(kGatherThreads), 0, pdl ? kPdl : kPlain, p);
   return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA;
@@ -474,7 +487,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // selection from candidates -> gather) needs the candidate lists and a selection small
 // enough for them; otherwise every score goes through the score workspace.
 bool use_candidates(const saga_ctx* h, int N) {
-  return h->cand_mask != nullptr && N <= kTopnSelNarrow && N <= kTopnCap / 4 && h->d <= kTopnMaxD &&
+  return h->cand_mask != nullptr && N <= kTopnSelNarrow && N <= kTopnCap / 4 && h->dv <= kTopnMaxD &&
          (N < h->max_seq_len || h->max_seq_len <= kTopnCap);
 }
 
@@ -542,6 +555,12 @@ const char* saga_decode_error_string(int code) {
 
 int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_q, int h_k,
                      int h_v, int head_dim, int max_N, void* cuda_stream) {
+  return saga_decode_init_kv(handle, max_batch, max_seq_len, h_q, h_k, h_v, head_dim, head_dim, max_N,
+                             cuda_stream);
+}
+
+int saga_decode_init_kv(saga_handle* handle, int max_batch, int max_seq_len, int h_q, int h_k,
+                        int h_v, int head_dim, int head_dim_v, int max_N, void* cuda_stream) {
   if (!handle) return SAGA_ERR_INVALID_ARG;
   *handle = nullptr;
   if (max_batch < 1 || max_batch > kMaxBatch) return SAGA_ERR_INVALID_ARG;
@@ -551,6 +570,7 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   if (static_cast<long long>(max_batch) * h_k * max_seq_len >= (1ll << 31)) return SAGA_ERR_INVALID_ARG;
   if (static_cast<long long>(max_batch) * h_q > (1ll << 30)) return SAGA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return SAGA_ERR_UNSUPPORTED;
+  if (head_dim_v != 64 && head_dim_v != 128) return SAGA_ERR_UNSUPPORTED;
   const int g = h_q / h_k;
   if (g > 64) return SAGA_ERR_UNSUPPORTED;
 
@@ -569,6 +589,7 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   h->max_batch = h->batch = max_batch;
   h->max_seq_len = max_seq_len;
   h->h_q = h_q; h->h_k = h_k; h->h_v = h_v; h->d = head_dim; h->max_N = max_N;
+  h->dv = head_dim_v;
   h->g = g; h->g_v = h_q / h_v;
   h->npad = round_up(g, 16);
   h->z_stride = round_up(max_seq_len, 32);
@@ -578,10 +599,10 @@ int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_len, int h_
   const size_t z_bytes = rows * h->z_stride * sizeof(float);
   const size_t stat_bytes = rows * sizeof(uint32_t);
   const size_t sel_bytes = rows * static_cast<size_t>(max_N) * 2 * 4;   // a step keeps up to 2N
-  const size_t qo_bytes = rows * head_dim * 2;
+  const size_t qo_bytes = rows * (head_dim > head_dim_v ? head_dim : head_dim_v) * 2;
   const int slots = max_N < max_seq_len ? max_N : max_seq_len;
   h->max_chunks = (slots + kGatherRows - 1) / kGatherRows;
-  const size_t part_bytes = rows * h->max_chunks * (head_dim + 2) * sizeof(float);
+  const size_t part_bytes = rows * h->max_chunks * (head_dim_v + 2) * sizeof(float);
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   // candidate path: chunk masks (the keys reuse z), sampled scores, bounds
   h->mask_stride = h->z_stride / 32;
@@ -661,6 +682,7 @@ int saga_atopn_calibrate(saga_handle h, const void* q, const void* k_cache, cons
                          void* out, int32_t* sel_idx, float* sel_logit, float* log_tau) {
   if (!h) return SAGA_ERR_INVALID_ARG;
   if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  if (h->dv != h->d) return SAGA_ERR_UNSUPPORTED;   // stateful Atop-N: one width
   return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit, kModeCalibrate,
                      log_tau);
 }
@@ -670,6 +692,7 @@ int saga_atopn_step(saga_handle h, const void* q, const void* k_cache, const voi
                     const float* log_tau, void* out, int32_t* sel_idx, float* sel_logit) {
   if (!h) return SAGA_ERR_INVALID_ARG;
   if (int rc = check_heads(h, h_q, h_k, h_v, head_dim)) return rc;
+  if (h->dv != h->d) return SAGA_ERR_UNSUPPORTED;   // stateful Atop-N: one width
   return decode_impl(h, q, k_cache, v_cache, seq_lens, N, out, sel_idx, sel_logit, kModeStep,
                      const_cast<float*>(log_tau));
 }
@@ -684,7 +707,7 @@ int saga_group_attn(saga_handle h, const void* q, const void* k_cache, const voi
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   // value groups inside key groups, every head of a key group in one epilogue warp,
   // the weights of N x g_v in the key list's shared memory
-  if (h->h_v % h->h_k != 0 || h->npad > 32 || h->g_v > kGroupMaxGv || N > kGroupMaxN ||
+  if (h->dv != h->d || h->h_v % h->h_k != 0 || h->npad > 32 || h->g_v > kGroupMaxGv || N > kGroupMaxN ||
       N * h->g_v > kTopnCap || !use_candidates(h, N))
     return SAGA_ERR_UNSUPPORTED;
   DeviceGuard dg(h->device);
@@ -717,8 +740,9 @@ int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;
-  const size_t qo = static_cast<size_t>(h->batch) * h->h_q * h->d * 2;
-  if (cudaMemcpyAsync(h->q_stage, q_host, qo, cudaMemcpyHostToDevice, h->stream) != cudaSuccess)
+  const size_t q_bytes = static_cast<size_t>(h->batch) * h->h_q * h->d * 2;
+  const size_t o_bytes = static_cast<size_t>(h->batch) * h->h_q * h->dv * 2;
+  if (cudaMemcpyAsync(h->q_stage, q_host, q_bytes, cudaMemcpyHostToDevice, h->stream) != cudaSuccess)
     return SAGA_ERR_CUDA;
   if (cudaMemcpyAsync(h->lens_stage, seq_lens_host, static_cast<size_t>(h->batch) * 4,
                       cudaMemcpyHostToDevice, h->stream) != cudaSuccess)
@@ -726,7 +750,7 @@ int saga_decode_attn_host(saga_handle h, const void* q_host, const void* k_cache
   int rc = decode_impl(h, h->q_stage, k_cache, v_cache, h->lens_stage, N, h->out_stage,
                        nullptr, nullptr);
   if (rc) return rc;
-  if (cudaMemcpyAsync(out_host, h->out_stage, qo, cudaMemcpyDeviceToHost, h->stream) != cudaSuccess)
+  if (cudaMemcpyAsync(out_host, h->out_stage, o_bytes, cudaMemcpyDeviceToHost, h->stream) != cudaSuccess)
     return SAGA_ERR_CUDA;
   return SAGA_OK;
 }
@@ -757,7 +781,7 @@ int saga_combine(saga_handle h, const int32_t* sel_idx, const float* sel_logit,
                  int N, void* out) {
   if (!h || !sel_idx || !sel_logit || !v_cache || !seq_lens || !out) return SAGA_ERR_INVALID_ARG;
   if (!aligned16(v_cache)) return SAGA_ERR_INVALID_ARG;
-  if (h_q != h->h_q || h_v != h->h_v || head_dim != h->d) return SAGA_ERR_INVALID_ARG;
+  if (h_q != h->h_q || h_v != h->h_v || head_dim != h->dv) return SAGA_ERR_INVALID_ARG;
   if (N < 1 || N > h->max_N) return SAGA_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);
   if (!dg.ok) return SAGA_ERR_CUDA;

@@ -112,8 +112,8 @@ struct TopnParams {
   float* log_tau;               // [B*h_q] written by calibration, read by a step
   int32_t* sel_idx;             // [B*h_q][cap]
   float* sel_logit;             // [B*h_q][cap]
-  const __nv_bfloat16* q;       // [B][h_q][D] (scoring a row again, fallback)
-  const __nv_bfloat16* k_cache; // [B][h_k][L_max][D]
+  const __nv_bfloat16* q;       // [B][h_q][DK] (scoring a row again, fallback)
+  const __nv_bfloat16* k_cache; // [B][h_k][L_max][DK]
   const __nv_bfloat16* v_cache; // [B][h_v][L_max][D]
   float scale;
   __nv_bfloat16* out;           // [B*h_q][D]
@@ -437,10 +437,12 @@ __device__ void topn_rescore(const __nv_bfloat16* q, const __nv_bfloat16* keys, 
 }
 
 // kMode: a TopnMode; kSel: the layout's selection capacity (>= the list width p.cap).
+// D: the value (and output) width; DK: the query and key width, used when a row
+// is scored again ("More Value per Key" §5.2 lets keys be narrower than values).
 // kRun: chunks per thread the shared-memory path takes (kTopnRun, or kTopnLongRun
 // for caches of more than 65536 positions; the longer variant costs the short
 // rows a few microseconds).
-template <int D, int kMode, int kSel, int kRun = kTopnRun>
+template <int D, int kMode, int kSel, int kRun = kTopnRun, int DK = D>
 __global__ void __launch_bounds__(kTopnThreads, 2)
 topn_kernel(const TopnParams p) {
   using Lay = TopnLayout<kSel>;
@@ -567,8 +569,8 @@ topn_kernel(const TopnParams p) {
   auto rescore = [&]() {
     if (tid == 0) atomicOr(p.status, 0x200 /* SAGA_STATUS_INFO_ROBUST_PATH */);
     const __nv_bfloat16* keys =
-        p.k_cache + (static_cast<long long>(b) * p.h_k + j / p.g) * p.L_max * D;
-    topn_rescore<D>(p.q + static_cast<long long>(bj) * D, keys, L, p.scale, krow);
+        p.k_cache + (static_cast<long long>(b) * p.h_k + j / p.g) * p.L_max * DK;
+    topn_rescore<DK>(p.q + static_cast<long long>(bj) * DK, keys, L, p.scale, krow);
     __syncthreads();                             // the row's keys are visible to the whole CTA
   };
 
