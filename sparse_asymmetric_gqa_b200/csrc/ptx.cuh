@@ -183,6 +183,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// The same for 64-byte rows with 64-byte swizzling (K-major): eight-row groups
+// 512 bytes apart, layout type 4.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(4u) << 61;
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, both K-major,
 // shape M x N.  Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16),
 // [10,13) B format (1 = bf16), 15/16 A/B major (0 = K), [17,23) N >> 3,

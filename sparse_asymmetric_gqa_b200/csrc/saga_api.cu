@@ -65,10 +65,13 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  // rows of 64 or more elements: 64-element boxes, 128-byte swizzle; 32-element
+  // rows (keys of width 32): one 64-byte box row, 64-byte swizzle
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(cols < 64 ? cols : 64), box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  cols < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -132,6 +135,7 @@ int set_smem_attrs_once() {
   if (e == cudaSuccess)                                                                           \
     e = cudaFuncSetAttribute(score_kernel<D, NP, true, true>,                                     \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreShape<D, NP>::kSmemBytes);
+    SAGA_ATTR(32, 16) SAGA_ATTR(32, 32) SAGA_ATTR(32, 48) SAGA_ATTR(32, 64)
     SAGA_ATTR(64, 16) SAGA_ATTR(64, 32) SAGA_ATTR(64, 48) SAGA_ATTR(64, 64)
     SAGA_ATTR(128, 16) SAGA_ATTR(128, 32) SAGA_ATTR(128, 48) SAGA_ATTR(128, 64)
 #undef SAGA_ATTR
@@ -165,7 +169,11 @@ int set_smem_attrs_once() {
                           reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnRun, 128>),
                           reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun, 128>),
                           reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnRun, 64>),
-                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun, 64>)})
+                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun, 64>),
+                          reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnRun, 32>),
+                          reinterpret_cast<const void*>(topn_kernel<64, kModeExact, kTopnSelNarrow, kTopnLongRun, 32>),
+                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnRun, 32>),
+                          reinterpret_cast<const void*>(topn_kernel<128, kModeExact, kTopnSelNarrow, kTopnLongRun, 32>)})
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(TopnLayout<kTopnSelNarrow>::kBytes));
@@ -254,6 +262,7 @@ int launch_score(saga_ctx* h, const void* q, const void* k_cache, const int32_t*
                       ScoreShape<D, NP>::kSmemBytes, kPdl, mk, mq, p, h->g_v)                          \
              : launch(h, score_kernel<D, NP, false>, dim3(grid), dim3(kScoreThreads),          \
                       ScoreShape<D, NP>::kSmemBytes, kPlain, mk, mq, p, h->g_v);
+  SAGA_CASE(32, 16) SAGA_CASE(32, 32) SAGA_CASE(32, 48) SAGA_CASE(32, 64)
   SAGA_CASE(64, 16) SAGA_CASE(64, 32) SAGA_CASE(64, 48) SAGA_CASE(64, 64)
   SAGA_CASE(128, 16) SAGA_CASE(128, 32) SAGA_CASE(128, 48) SAGA_CASE(128, 64)
 #undef SAGA_CASE
@@ -291,7 +300,9 @@ int launch_bounds(saga_ctx* h, const void* q, const void* k_cache, const int32_t
   p.m_ref = ref ? h->m_ref : nullptr;
   const dim3 sgrid(h->batch * h->h_k, kSampleParts);
   const size_t smem = static_cast<size_t>(h->g) * h->d * sizeof(float);
-  cudaError_t e = (h->d == 64)
+  cudaError_t e = (h->d == 32)
+      ? launch(h, sample_kernel<32>, sgrid, dim3(kSampleThreads), smem, kPlain, p)
+      : (h->d == 64)
       ? launch(h, sample_kernel<64>, sgrid, dim3(kSampleThreads), smem, kPlain, p)
       : launch(h, sample_kernel<128>, sgrid, dim3(kSampleThreads), smem, kPlain, p);
   if (e == cudaSuccess) e = launch(h, bound_kernel, dim3(h->batch * h->h_q), dim3(32), 0, kPdl, p);
@@ -337,8 +348,10 @@ int launch_topn(saga_ctx* h, const void* q, const void* k_cache, const void* v_c
     const bool long_rows = h->max_seq_len > kTopnThreads * 32 * kTopnRun;
     if (h->dv == 64 && h->d == 64) e = launch_topn_exact<64, 64>(h, grid, block, narrow, p, long_rows);
     else if (h->dv == 128 && h->d == 128) e = launch_topn_exact<128, 128>(h, grid, block, narrow, p, long_rows);
-    else if (h->dv == 128) e = launch_topn_exact<128, 64>(h, grid, block, narrow, p, long_rows);
-    else e = launch_topn_exact<64, 128>(h, grid, block, narrow, p, long_rows);
+    else if (h->dv == 128 && h->d == 64) e = launch_topn_exact<128, 64>(h, grid, block, narrow, p, long_rows);
+    else if (h->dv == 64 && h->d == 128) e = launch_topn_exact<64, 128>(h, grid, block, narrow, p, long_rows);
+    else if (h->dv == 128) e = launch_topn_exact<128, 32>(h, grid, block, narrow, p, long_rows);
+    else e = launch_topn_exact<64, 32>(h, grid, block, narrow, p, long_rows);
   } else if (mode == kModeCalibrate)
     e = (h->d == 64) ? launch(h, topn_kernel<64, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p)
                      : launch(h, topn_kernel<128, kModeCalibrate, kTopnSelNarrow>, grid, block, narrow, kPdl, p);
@@ -569,7 +582,7 @@ int saga_decode_init_kv(saga_handle* handle, int max_batch, int max_seq_len, int
   if (h_q % h_k != 0 || h_q % h_v != 0) return SAGA_ERR_INVALID_ARG;
   if (static_cast<long long>(max_batch) * h_k * max_seq_len >= (1ll << 31)) return SAGA_ERR_INVALID_ARG;
   if (static_cast<long long>(max_batch) * h_q > (1ll << 30)) return SAGA_ERR_INVALID_ARG;
-  if (head_dim != 64 && head_dim != 128) return SAGA_ERR_UNSUPPORTED;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return SAGA_ERR_UNSUPPORTED;
   if (head_dim_v != 64 && head_dim_v != 128) return SAGA_ERR_UNSUPPORTED;
   const int g = h_q / h_k;
   if (g > 64) return SAGA_ERR_UNSUPPORTED;

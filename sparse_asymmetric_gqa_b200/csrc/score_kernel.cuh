@@ -62,11 +62,15 @@ struct ScoreParams {
 
 template <int D, int NPAD>
 struct ScoreShape {
-  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(D == 32 || D == 64 || D == 128, "head_dim");
   static_assert(NPAD % 16 == 0 && NPAD >= 16 && NPAD <= 64, "padded group");
-  static constexpr int kParts = D / 64;                 // 128-byte swizzle atoms along d
-  static constexpr int kAPart = kTileM * 128;           // 16 KB of K per atom
-  static constexpr int kBPart = NPAD * 128;             // q rows per atom
+  // swizzle atoms along d: rows of 64 elements (128-byte swizzle), or of 32
+  // elements for d = 32 (64-byte swizzle)
+  static constexpr int kAtomElems = D < 64 ? D : 64;
+  static constexpr int kAtomBytes = kAtomElems * 2;
+  static constexpr int kParts = D / kAtomElems;
+  static constexpr int kAPart = kTileM * kAtomBytes;    // K rows per atom (16 KB, or 8 KB for d = 32)
+  static constexpr int kBPart = NPAD * kAtomBytes;      // q rows per atom
   static constexpr int kStageBytes = kParts * (kAPart + kBPart);
   // 128 KB of K in flight per SM (four stages for d = 128) measured faster than
   // 160 or 192 KB: more bytes in flight only lengthened the memory queues.
@@ -268,10 +272,10 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t bq = a + S::kParts * S::kAPart;
 #pragma unroll
         for (int part = 0; part < S::kParts; ++part)
-          tma_load_2d(a + part * S::kAPart, &tmap_k, part * 64, row, full_bar(s), pol_k);
+          tma_load_2d(a + part * S::kAPart, &tmap_k, part * S::kAtomElems, row, full_bar(s), pol_k);
 #pragma unroll
         for (int part = 0; part < S::kParts; ++part)
-          tma_load_2d(bq + part * S::kBPart, &tmap_q, part * 64, qrow, full_bar(s), pol_q);
+          tma_load_2d(bq + part * S::kBPart, &tmap_q, part * S::kAtomElems, qrow, full_bar(s), pol_q);
       }
       // Let every load this thread issued land before the CTA can exit.
       const int first = i > S::kStages ? i - S::kStages : 0;
@@ -298,10 +302,14 @@ score_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t d_tmem = tmem_base + buf * S::kAccStride;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int part = k >> 2;
-          const uint32_t off = (k & 3) * 32;   // 16 bf16 = 32 bytes along the swizzled row
-          tc_mma_bf16(d_tmem, smem_desc_sw128(a + part * S::kAPart + off),
-                      smem_desc_sw128(bq + part * S::kBPart + off), idesc, k > 0 ? 1u : 0u);
+          constexpr int kSteps = S::kAtomElems / 16;   // MMAs per atom row
+          const int part = k / kSteps;
+          const uint32_t off = (k % kSteps) * 32;     // 16 bf16 = 32 bytes along the swizzled row
+          const uint32_t da = a + part * S::kAPart + off, db = bq + part * S::kBPart + off;
+          if constexpr (S::kAtomBytes == 128)
+            tc_mma_bf16(d_tmem, smem_desc_sw128(da), smem_desc_sw128(db), idesc, k > 0 ? 1u : 0u);
+          else
+            tc_mma_bf16(d_tmem, smem_desc_sw64(da), smem_desc_sw64(db), idesc, k > 0 ? 1u : 0u);
         }
         tc_commit(empty_bar(s));
         tc_commit(accf_bar(buf));

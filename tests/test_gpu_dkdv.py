@@ -1,7 +1,8 @@
 """Keys and values of different widths ("More Value per Key" §5.2) on the GPU.
 
 A handle made with ``head_dim_v`` != ``head_dim`` scores with the key width
-(scale 1/sqrt(d_k)) and gathers values of the value width.  Every row is checked
+(scale 1/sqrt(d_k)) and gathers values of the value width; keys of width 32 (the
+pages' (h_k, d_k) = (2, 32) variant) take the score pass's 64-byte-swizzle tiles.  Every row is checked
 against the oracle with the rules of ``parity_utils`` (scores with d_k terms,
 outputs of width d_v), on the candidate path (N <= 2048 and short of the row)
 and on the score-row path (N >= L_b: every position).
@@ -23,7 +24,7 @@ def make_kv(seed, B, L, lens, h_q, h_k, h_v, d_k, d_v):
     return workload.DecodeInputs(q, k, v, torch.tensor(lens, dtype=torch.int32))
 
 
-@pytest.mark.parametrize("d_k,d_v", [(64, 128), (128, 64)])
+@pytest.mark.parametrize("d_k,d_v", [(64, 128), (128, 64), (32, 64), (32, 128)])
 @pytest.mark.parametrize("case", [
     # (B, L, lens, h_q, h_k, h_v, N)
     (3, 20000, [20000, 9000, 777], 8, 2, 4, 512),     # candidate path, ragged rows
