@@ -102,8 +102,8 @@ SAGA_API int saga_decode_init(saga_handle* handle, int max_batch, int max_seq_le
                      int h_q, int h_k, int h_v, int head_dim, int max_N,
                      void* cuda_stream);
 
-/* As saga_decode_init, with keys (and queries) of width head_dim and values (and
- * outputs) of width head_dim_v, each 64 or 128 ("More Value per Key" §5.2: keys
+/* As saga_decode_init, with keys (and queries) of width head_dim (32, 64 or 128)
+ * and values (and outputs) of width head_dim_v (64 or 128) ("More Value per Key" §5.2: keys
  * narrower than values; the scale stays 1/sqrt(head_dim)).  On such a handle the
  * head_dim argument of every call is the key width; q is [B][h_q][head_dim],
  * k_cache [B][h_k][L_max][head_dim], v_cache [B][h_v][L_max][head_dim_v], out
