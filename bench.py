@@ -52,9 +52,11 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--workload", default="qwen32k",
-                    choices=["qwen32k", "dense_llama", "llama_ragged", "sweep"],
+                    choices=["qwen32k", "qwen32k_call", "dense_llama", "llama_ragged", "qwen32k_dk32",
+                             "sweep"],
                     help="qwen32k: the headline line (default); the others print one line of "
-                         "per-call throughput for that workload (the sweep: one line, 27 points)")
+                         "per-call throughput for that workload (qwen32k_call: the headline's "
+                         "workload timed call by call; the sweep: one line, 27 points)")
     ap.add_argument("--layers", type=int, default=None,
                     help="layers per step (default: the workload's 28); fewer only for small "
                          "profiling captures, never for a reported number")
@@ -294,9 +296,9 @@ def time_workload(spec, dev, steps, warmup, flush):
     from sparse_asymmetric_gqa_b200 import SagaDecoder, workload
     x = workload.make_inputs(spec, layer=0, device=dev)
     B = spec.batch
-    out = torch.empty(B, spec.h_q, spec.head_dim, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(B, spec.h_q, spec.d_v, dtype=torch.bfloat16, device=dev)
     dec = SagaDecoder(B, spec.seq_len, spec.h_q, spec.h_k, spec.h_v, spec.head_dim, spec.N,
-                      device=dev)
+                      device=dev, head_dim_v=spec.d_v)
     dec.attn(x.q, x.k_cache, x.v_cache, x.seq_lens, spec.N, out=out)
     status = dec.status()
     if status & 0xFF:
@@ -326,7 +328,7 @@ def time_workload(spec, dev, steps, warmup, flush):
     times = sorted(a.elapsed_time(b) for a, b in ev)
     lens = [int(v) for v in x.seq_lens.tolist()]
     k_bytes = sum(spec.h_k * Lb * spec.head_dim * 2 for Lb in lens)
-    v_bytes = sum(spec.h_v * min(spec.N, Lb) * spec.head_dim * 2 for Lb in lens)
+    v_bytes = sum(spec.h_v * min(spec.N, Lb) * spec.d_v * 2 for Lb in lens)
     del graph, dec, x
     torch.cuda.empty_cache()
     return {"ms_mean": sum(times) / len(times), "ms_median": times[len(times) // 2],
@@ -341,7 +343,9 @@ def run_workloads(args, rank, world, local):
     if args.workload == "sweep":
         specs = workload.sweep_specs()
     else:
-        specs = [{"dense_llama": workload.DENSE_LLAMA, "llama_ragged": workload.LLAMA_RAGGED}[args.workload]]
+        specs = [{"dense_llama": workload.DENSE_LLAMA, "llama_ragged": workload.LLAMA_RAGGED,
+                  "qwen32k_dk32": workload.QWEN_32K_DK32,
+                  "qwen32k_call": workload.QWEN_32K}[args.workload]]
     flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)     # 256 MB > 126 MB L2
     peak, peak_src = measured_hbm_peak()
     steps = max(3, min(args.steps, 20))
@@ -353,7 +357,7 @@ def run_workloads(args, rank, world, local):
         points.append({
             "workload": spec.name, "batch": spec.batch, "seq_len": spec.seq_len, "N": spec.N,
             "h_q": spec.h_q, "h_k": spec.h_k, "h_v": spec.h_v, "head_dim": spec.head_dim,
-            "ragged": spec.ragged, "tokens_per_s": world * spec.batch / call_s,
+            "head_dim_v": spec.d_v, "ragged": spec.ragged, "tokens_per_s": world * spec.batch / call_s,
             "calls_per_s": world / call_s, "ms_per_call": call_s * 1e3,
             "ms_per_call_median": r["ms_median"], "gpu_launches_per_call": r["launches"],
             "model_bytes_per_call": r["k_bytes"] + r["v_bytes_model"], "achieved_gbs": gbs,

@@ -38,6 +38,11 @@ class DecodeSpec:
     ragged: Optional[Tuple[int, int]] = None  # seq_lens ~ U{lo..hi} if set
     layers: int = 1
     seed: int = 0
+    head_dim_v: Optional[int] = None          # value width when it differs from head_dim
+
+    @property
+    def d_v(self) -> int:
+        return self.head_dim if self.head_dim_v is None else self.head_dim_v
 
     @property
     def g(self) -> int:
@@ -81,7 +86,14 @@ def sweep_specs():
     return out
 
 
-CONFIGS = {s.name: s for s in (TINY, DENSE_LLAMA, QWEN_32K, LLAMA_RAGGED)}
+# The pages' key-dimension variant of the Qwen shape ("More Value per Key" §5.2):
+# (h_k, d_k) = (2, 32) with full-width values, so the key cache is half of the
+# merged h_k = 1, d = 128 one.
+QWEN_32K_DK32 = DecodeSpec("qwen2.5-1.5b_b16_l32k_n1024_hk2_dk32", batch=16, seq_len=32768, h_q=12,
+                           h_k=2, h_v=2, head_dim=32, N=1024, planted_frac=0.02,
+                           plant_scale=(2.0, 4.0), seed=3500, head_dim_v=128)
+
+CONFIGS = {s.name: s for s in (TINY, DENSE_LLAMA, QWEN_32K, LLAMA_RAGGED, QWEN_32K_DK32)}
 
 
 @dataclass
@@ -109,7 +121,7 @@ def make_inputs(spec: DecodeSpec, layer: int = 0, device="cpu",
 
     q = randn(B, spec.h_q, d)
     k_cache = randn(B, spec.h_k, L, d)
-    v_cache = randn(B, spec.h_v, L, d)
+    v_cache = randn(B, spec.h_v, L, spec.d_v)
     if spec.ragged is not None:
         lo, hi = spec.ragged
         seq_lens = torch.randint(lo, hi + 1, (B,), generator=gen, device=dev,
