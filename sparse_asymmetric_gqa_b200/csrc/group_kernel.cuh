@@ -234,33 +234,72 @@ group_kernel(const GroupParams p) {
       listp = false;
     } else {
       listp = C <= static_cast<uint32_t>(kGroupCap) && fits;
-      uint32_t o = off;
-      // a chunk's kept positions hold their keys at consecutive slots: the keys of
-      // kGroupBlock positions (all heads) are loaded before any of them is used
-      for (int c = c0; c < c1; ++c) {
-        uint32_t m = __ldcg(mrow + c);
-        const int n_c = __popc(m);
-        const uint32_t* ac = area + static_cast<long long>(c) * 32 * g_v;
-        for (int k0 = 0; k0 < n_c; k0 += kGroupBlock) {
-          uint32_t kv[kGroupBlock][kGroupMaxGv];
-#pragma unroll
-          for (int u = 0; u < kGroupBlock; ++u)
-#pragma unroll
-            for (int e = 0; e < kGroupMaxGv; ++e)
-              kv[u][e] = (k0 + u < n_c && e < g_v) ? __ldcg(ac + (k0 + u) * g_v + e) : 0u;
+      if (listp) {
+        // the list in position order: each thread expands its chunks' masks into
+        // positions and key slots (slot = 32 c + rank in the chunk; s_key holds the
+        // slot until s replaces it), then s of entry i is formed by thread i mod 256,
+        // so a warp reads the keys of 32 consecutive entries, mostly consecutive slots
+        uint32_t o = off;
+        for (int c = c0; c < c1; ++c) {
+          uint32_t m = __ldcg(mrow + c);
+          const int n_c = __popc(m);
+          for (int k = 0; k < n_c; ++k) {
+            s_pos[o] = c * 32 + (__ffs(m) - 1);
+            s_key[o] = static_cast<uint32_t>(c * 32 + k);
+            m &= m - 1u;
+            ++o;
+          }
+        }
+        __syncthreads();
+        for (int i0 = 0; i0 < static_cast<int>(C); i0 += kTopnThreads * kGroupBlock) {
+          uint32_t slot[kGroupBlock], kv[kGroupBlock][kGroupMaxGv];
 #pragma unroll
           for (int u = 0; u < kGroupBlock; ++u) {
-            if (k0 + u < n_c) {
-              const int pos = c * 32 + (__ffs(m) - 1);
-              m &= m - 1u;
-              float s = 0.0f;
+            const int i = i0 + u * kTopnThreads + tid;
+            slot[u] = i < static_cast<int>(C) ? s_key[i] : 0u;
+#pragma unroll
+            for (int e = 0; e < kGroupMaxGv; ++e)
+              kv[u][e] = (i < static_cast<int>(C) && e < g_v)
+                             ? __ldcg(area + static_cast<long long>(slot[u]) * g_v + e) : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < kGroupBlock; ++u) {
+            const int i = i0 + u * kTopnThreads + tid;
+            if (i < static_cast<int>(C)) {
+              float sv = 0.0f;
 #pragma unroll
               for (int e = 0; e < kGroupMaxGv; ++e)
-                if (e < g_v) s += expf(key_to_float(kv[u][e]) - lse[e]);
-              const uint32_t key = ordered_key(s);
-              srow[c * 32 + k0 + u] = key;
-              if (listp) { s_key[o] = key; s_pos[o] = pos; }
-              ++o;
+                if (e < g_v) sv += expf(key_to_float(kv[u][e]) - lse[e]);
+              const uint32_t key = ordered_key(sv);
+              srow[slot[u]] = key;
+              s_key[i] = key;
+            }
+          }
+        }
+      } else {                                   // the slots in global memory: s per chunk
+        // a chunk's kept positions hold their keys at consecutive slots: the keys of
+        // kGroupBlock positions (all heads) are loaded before any of them is used
+        for (int c = c0; c < c1; ++c) {
+          uint32_t m = __ldcg(mrow + c);
+          const int n_c = __popc(m);
+          const uint32_t* ac = area + static_cast<long long>(c) * 32 * g_v;
+          for (int k0 = 0; k0 < n_c; k0 += kGroupBlock) {
+            uint32_t kv[kGroupBlock][kGroupMaxGv];
+#pragma unroll
+            for (int u = 0; u < kGroupBlock; ++u)
+#pragma unroll
+              for (int e = 0; e < kGroupMaxGv; ++e)
+                kv[u][e] = (k0 + u < n_c && e < g_v) ? __ldcg(ac + (k0 + u) * g_v + e) : 0u;
+#pragma unroll
+            for (int u = 0; u < kGroupBlock; ++u) {
+              if (k0 + u < n_c) {
+                float s = 0.0f;
+#pragma unroll
+                for (int e = 0; e < kGroupMaxGv; ++e)
+                  if (e < g_v) s += expf(key_to_float(kv[u][e]) - lse[e]);
+                const uint32_t key = ordered_key(s);
+                srow[c * 32 + k0 + u] = key;
+              }
             }
           }
         }
